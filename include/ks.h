@@ -1,0 +1,138 @@
+/*
+ * ks.h -- C ABI of the B200 (sm_100a) library for multiplication by
+ * Kronecker-sparse (KS) matrices.
+ *
+ * The operation (taxoreview.com page on Kronecker-sparse matrix
+ * multiplication, first abstract: KS supports are Kronecker products of
+ * identity and all-ones blocks; butterfly and Monarch matrices are products of
+ * KS factors).  Read with the textbook Kronecker index order, a KS factor of
+ * pattern (a, b, c, d) is the (a*b*d) x (a*c*d) matrix K with support
+ * I_a (x) 1_{b x c} (x) I_d,
+ *
+ *     K[i*b*d + k*d + l][i*c*d + j*d + l] = values[i][l][k][j],
+ *     i < a, k < b, j < c, l < d,
+ *
+ * and the library computes, for a batch of `batch` rows,
+ *
+ *     Y[n][i*b*d + k*d + l] = sum_{j<c} values[i][l][k][j] * X[n][i*c*d + j*d + l],
+ *
+ * i.e. Y = X * K^T, without ever forming K and without permutation kernels.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named X, values, factors[t], Y are DEVICE pointers (memory of
+ *     the current CUDA device), owned by the caller.  The library keeps none
+ *     of them after the call returns and frees nothing it did not allocate.
+ *   - X is batch x (a*c*d) row-major; Y is batch x (a*b*d) row-major;
+ *     values is the contiguous array values[a][d][b][c].
+ *   - X, values and Y share one storage type: fp32 for KS_F32 and KS_TF32,
+ *     bf16 for KS_BF16 (Y is written in bf16, rounded to nearest even from an
+ *     fp32 accumulator).  KS_TF32 reads fp32 buffers and multiplies in TF32
+ *     (accumulating in fp32); it is never chosen silently for KS_F32.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on that stream; the return value reports only
+ *     errors found before or at launch.  Errors found on the device (a bounded
+ *     wait that gave up) are reported by ks_sync_status().
+ *   - Y must not overlap X or values (KS_ERR_INVALID_ARG).
+ *   - batch == 0 is a no-op returning KS_OK.  Negative or zero pattern
+ *     entries, negative batch, or sizes whose element counts overflow int64
+ *     return KS_ERR_INVALID_ARG.  Any pointer alignment is accepted (fp32
+ *     needs 4-byte, bf16 2-byte alignment at least, else KS_ERR_MISALIGNED);
+ *     16-byte aligned pointers and row widths take the vectorised kernels.
+ *   - No exception crosses this interface.  All calls are thread-safe; the
+ *     message of the last failing call is kept per host thread.
+ */
+#ifndef KS_B200_KS_H
+#define KS_B200_KS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage / arithmetic type of X, values and Y. */
+typedef enum ks_dtype {
+    KS_F32 = 0,  /* fp32 storage, fp32 FMA arithmetic                         */
+    KS_TF32 = 1, /* fp32 storage, TF32 tensor-core products, fp32 accumulate  */
+    KS_BF16 = 2  /* bf16 storage, bf16 tensor-core products, fp32 accumulate  */
+} ks_dtype;
+
+typedef enum ks_status {
+    KS_OK = 0,
+    KS_ERR_INVALID_ARG = 1, /* bad pattern, batch, dtype, pointer or overlap          */
+    KS_ERR_MISALIGNED = 2,  /* pointer not aligned to its element size                */
+    KS_ERR_UNSUPPORTED = 3, /* variant forced on a pattern it cannot run              */
+    KS_ERR_ALLOC = 4,       /* workspace allocation failed (ks_chain)                 */
+    KS_ERR_CUDA = 5,        /* a CUDA runtime call failed; see ks_last_error()        */
+    KS_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (ks_sync_status)    */
+} ks_status;
+
+/* Kernel families.  KS_VARIANT_AUTO lets the library's pattern heuristic
+ * choose; the others force one family (for tests and measurements). */
+typedef enum ks_variant {
+    KS_VARIANT_AUTO = 0,
+    KS_VARIANT_STREAM = 1, /* bandwidth kernel: each thread reads its c inputs
+                              directly; any pattern, meant for b, c <= 8      */
+    KS_VARIANT_FMA = 2,    /* output-stationary CUDA-core gather-GEMM          */
+    KS_VARIANT_TC = 3      /* tcgen05 tensor-core block-GEMM (TF32 / BF16)     */
+} ks_variant;
+
+/* One factor's pattern: K is (a*b*d) x (a*c*d) with support I_a (x) 1_{b x c} (x) I_d. */
+typedef struct ks_pattern {
+    int64_t a, b, c, d;
+} ks_pattern;
+
+/* Y = X * K^T for one KS factor (see the top of this file for the layout).
+ * dtype is a ks_dtype; stream a cudaStream_t.  The pattern heuristic picks the
+ * kernel. */
+ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
+                    int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
+                    void *stream);
+
+/* ks_matmul with the kernel family forced (a ks_variant).  Returns
+ * KS_ERR_UNSUPPORTED if that family cannot run this pattern / dtype /
+ * alignment (e.g. KS_VARIANT_TC with dtype KS_F32). */
+ks_status ks_matmul_variant(const void *X, const void *values, int64_t a,
+                            int64_t b, int64_t c, int64_t d, int64_t batch,
+                            void *Y, int dtype, int variant, void *stream);
+
+/* What KS_VARIANT_AUTO would run for this problem, written to *variant
+ * (a ks_variant).  Host-only: touches no device. */
+ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
+                  int dtype, int *variant);
+
+/* A chain of KS factors applied in order, factor 0 first:
+ *     Y = X * (K_{n-1} ... K_1 K_0)^T.
+ * factors is a HOST array of n_factors DEVICE pointers, factor t holding
+ * values[a_t][d_t][b_t][c_t]; patterns is a HOST array of n_factors patterns.
+ * Widths must chain: a_t*b_t*d_t == a_{t+1}*c_{t+1}*d_{t+1}, else
+ * KS_ERR_INVALID_ARG.  X is batch x (a_0*c_0*d_0), Y is
+ * batch x (a_{n-1}*b_{n-1}*d_{n-1}).  Intermediates (in the chain's storage
+ * dtype) live in two workspace buffers allocated stream-ordered
+ * (cudaMallocAsync) and freed on the same stream before return
+ * (KS_ERR_ALLOC if that fails).  Each factor runs the kernel the pattern
+ * heuristic picks. */
+ks_status ks_chain(const void *X, const void *const *factors,
+                   const ks_pattern *patterns, int n_factors, int64_t batch,
+                   void *Y, int dtype, void *stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char *ks_last_error(void);
+
+/* Static name of a status code. */
+const char *ks_status_string(int status);
+
+/* Synchronises `stream`, then reports (and clears) the device-side status
+ * word of the current device: KS_ERR_TIMEOUT if a bounded wait inside a
+ * kernel gave up since the last call, KS_ERR_CUDA if the stream itself
+ * failed, KS_OK otherwise. */
+ks_status ks_sync_status(void *stream);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ks_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KS_B200_KS_H */

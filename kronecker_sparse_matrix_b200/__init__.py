@@ -1,0 +1,111 @@
+"""B200 (sm_100a) library for multiplication by Kronecker-sparse (KS) matrices.
+
+Y = X K^T with K of pattern (a, b, c, d), support I_a (x) 1_{b x c} (x) I_d
+and values[a][d][b][c], for one factor (``matmul``) or a chain of factors
+(``chain``) -- the operation of the taxoreview.com page on Kronecker-sparse
+matrix multiplication (first abstract).  Every step runs in the CUDA kernels
+of ``libks_b200.so`` behind the C ABI of ``include/ks.h``; this module only
+marshals torch tensors (device memory and streams) into that ABI.  There is no
+CPU or PyTorch fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import (KS_BF16, KS_F32, KS_TF32, KS_VARIANT_AUTO, KS_VARIANT_FMA,  # noqa: F401
+                   KS_VARIANT_STREAM, KS_VARIANT_TC, KsError, KsPattern, VARIANTS)
+
+Pattern = Tuple[int, int, int, int]
+
+__all__ = ["matmul", "chain", "plan", "sync_status", "ks_dtype_of", "KsError", "VARIANTS"]
+
+
+def ks_dtype_of(t: torch.Tensor, tf32: bool = False) -> int:
+    if t.dtype == torch.float32:
+        return KS_TF32 if tf32 else KS_F32
+    if t.dtype == torch.bfloat16:
+        if tf32:
+            raise ValueError("tf32 applies to fp32 tensors only")
+        return KS_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: use float32 or bfloat16")
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _variant(v) -> int:
+    if isinstance(v, str):
+        return VARIANTS[v]
+    return int(v)
+
+
+def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Optional[torch.Tensor] = None,
+           tf32: bool = False, variant="auto", stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Y = X K^T for one KS factor.  x: (batch, a*c*d) CUDA tensor (fp32 or
+    bf16), values: a*b*c*d entries in [a][d][b][c] order, same dtype/device.
+    Asynchronous on ``stream`` (default: the current stream)."""
+    a, b, c, d = (int(v) for v in pattern)
+    lib = _lib.load()
+    if x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D CUDA tensor")
+    if not (x.is_contiguous() and values.is_contiguous()):
+        raise ValueError("x and values must be contiguous")
+    if values.dtype != x.dtype or values.device != x.device:
+        raise ValueError("values must match x in dtype and device")
+    dt = ks_dtype_of(x, tf32)
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, a * b * d), dtype=x.dtype, device=x.device)
+    elif not out.is_contiguous() or out.dtype != x.dtype or out.device != x.device:
+        raise ValueError("out must be contiguous with x's dtype and device")
+    with torch.cuda.device(x.device):
+        st = lib.ks_matmul_variant(x.data_ptr(), values.data_ptr(), a, b, c, d, batch, out.data_ptr(), dt,
+                                   _variant(variant), _stream_ptr(stream, x.device))
+    _lib.check(st)
+    return out
+
+
+def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[Pattern], *,
+          out: Optional[torch.Tensor] = None, tf32: bool = False,
+          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Y = X (K_{n-1} ... K_0)^T, factor 0 applied first."""
+    lib = _lib.load()
+    n = len(factors)
+    if n == 0 or len(patterns) != n:
+        raise ValueError("need one pattern per factor")
+    if x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D CUDA tensor")
+    for f in factors:
+        if f.dtype != x.dtype or f.device != x.device or not f.is_contiguous():
+            raise ValueError("factors must be contiguous, with x's dtype and device")
+    dt = ks_dtype_of(x, tf32)
+    a, b, c, d = (int(v) for v in patterns[-1])
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, a * b * d), dtype=x.dtype, device=x.device)
+    ptrs = (ctypes.c_void_p * n)(*[f.data_ptr() for f in factors])
+    pats = (KsPattern * n)(*[KsPattern(*[int(v) for v in p]) for p in patterns])
+    with torch.cuda.device(x.device):
+        st = lib.ks_chain(x.data_ptr(), ptrs, pats, n, batch, out.data_ptr(), dt, _stream_ptr(stream, x.device))
+    _lib.check(st)
+    return out
+
+
+def plan(pattern: Pattern, batch: int, dtype: int = KS_F32) -> str:
+    """Name of the kernel family the heuristic picks (host only)."""
+    v = ctypes.c_int(-1)
+    a, b, c, d = (int(t) for t in pattern)
+    _lib.check(_lib.load().ks_plan(a, b, c, d, int(batch), int(dtype), ctypes.byref(v)))
+    return {v_: k for k, v_ in VARIANTS.items()}[v.value]
+
+
+def sync_status(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Synchronise and raise KsError if a kernel reported a device-side failure."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _lib.check(_lib.load().ks_sync_status(_stream_ptr(stream, dev)))

@@ -1,0 +1,298 @@
+// C ABI of the KS library: argument validation, dispatch to a kernel family,
+// the chain executor and error reporting.  Everything here runs on the host;
+// the only device work is the kernels the launchers enqueue and the chain's
+// stream-ordered workspace.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "ks.h"
+#include "ks_internal.h"
+
+namespace ks {
+namespace {
+
+thread_local char g_msg[512] = "";
+
+ks_status fail(ks_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ks_status ok() { return KS_OK; }
+
+// a*b with overflow check on non-negative operands.
+bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+bool ranges_overlap(const void *p, int64_t pbytes, const void *q, int64_t qbytes) {
+    if (!p || !q || pbytes <= 0 || qbytes <= 0) return false;
+    auto a0 = reinterpret_cast<uintptr_t>(p), b0 = reinterpret_cast<uintptr_t>(q);
+    return a0 < b0 + (uintptr_t)qbytes && b0 < a0 + (uintptr_t)pbytes;
+}
+
+// Validates one factor's sizes; fills the element counts.
+ks_status check_sizes(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
+                      int64_t *in_f, int64_t *out_f, int64_t *nvals) {
+    if (a <= 0 || b <= 0 || c <= 0 || d <= 0)
+        return fail(KS_ERR_INVALID_ARG, "pattern entries must be positive (a=%lld b=%lld c=%lld d=%lld)",
+                    (long long)a, (long long)b, (long long)c, (long long)d);
+    if (batch < 0) return fail(KS_ERR_INVALID_ARG, "batch must be >= 0 (got %lld)", (long long)batch);
+    int64_t ac, acd, ab, abd, abc, abcd, t1, t2;
+    if (!mul_ok(a, c, &ac) || !mul_ok(ac, d, &acd) || !mul_ok(a, b, &ab) || !mul_ok(ab, d, &abd) ||
+        !mul_ok(ab, c, &abc) || !mul_ok(abc, d, &abcd) || !mul_ok(std::max<int64_t>(batch, 1), acd, &t1) ||
+        !mul_ok(std::max<int64_t>(batch, 1), abd, &t2) || !mul_ok(t1, 4, &t1) || !mul_ok(t2, 4, &t2) ||
+        !mul_ok(abcd, 4, &abcd))
+        return fail(KS_ERR_INVALID_ARG, "sizes overflow int64");
+    // the kernels index rows with 32-bit feature offsets
+    if (acd > INT32_MAX || abd > INT32_MAX || abcd / 4 > INT32_MAX)
+        return fail(KS_ERR_INVALID_ARG, "a row or the values array exceeds 2^31 elements");
+    *in_f = acd;
+    *out_f = abd;
+    *nvals = abcd / 4;
+    return KS_OK;
+}
+
+ks_status check_dtype(int dtype) {
+    if (dtype != KS_F32 && dtype != KS_TF32 && dtype != KS_BF16)
+        return fail(KS_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    return KS_OK;
+}
+
+ks_status check_align(const void *p, int elem, const char *name) {
+    if (reinterpret_cast<uintptr_t>(p) % (uintptr_t)elem != 0)
+        return fail(KS_ERR_MISALIGNED, "%s is not aligned to its %d-byte element", name, elem);
+    return KS_OK;
+}
+
+ks_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(KS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Validates a single product and builds the Problem; *noop set for batch == 0.
+ks_status make_problem(const void *X, const void *V, int64_t a, int64_t b, int64_t c, int64_t d,
+                       int64_t batch, void *Y, int dtype, void *stream, Problem *p, bool *noop) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    int64_t in_f, out_f, nvals;
+    if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
+    *noop = (batch == 0);
+    if (*noop) return KS_OK;
+    if (!X || !V || !Y) return fail(KS_ERR_INVALID_ARG, "X, values and Y must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    if ((s = check_align(X, elem, "X")) != KS_OK) return s;
+    if ((s = check_align(V, elem, "values")) != KS_OK) return s;
+    if ((s = check_align(Y, elem, "Y")) != KS_OK) return s;
+    const int64_t ybytes = batch * out_f * elem;
+    if (ranges_overlap(Y, ybytes, X, batch * in_f * elem))
+        return fail(KS_ERR_INVALID_ARG, "Y overlaps X");
+    if (ranges_overlap(Y, ybytes, V, nvals * elem))
+        return fail(KS_ERR_INVALID_ARG, "Y overlaps values");
+    *p = Problem{X, V, Y, a, b, c, d, batch, dtype, static_cast<cudaStream_t>(stream)};
+    return KS_OK;
+}
+
+ks_status run(const Problem &p, int variant) {
+    Plan plan;
+    const char *why = "";
+    if (!make_plan(p, variant, &plan, &why))
+        return fail(KS_ERR_UNSUPPORTED, "variant %d cannot run pattern (%lld,%lld,%lld,%lld) dtype %d: %s",
+                    variant, (long long)p.a, (long long)p.b, (long long)p.c, (long long)p.d, p.dtype, why);
+    cudaError_t e = cudaSuccess;
+    switch (plan.variant) {
+        case KS_VARIANT_STREAM: e = launch_stream(p); break;
+        case KS_VARIANT_FMA: e = launch_fma(p, plan.fma); break;
+        case KS_VARIANT_TC: e = launch_tc(p, plan.tc); break;
+        default: return fail(KS_ERR_UNSUPPORTED, "no kernel for variant %d", plan.variant);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return ok();
+}
+
+// Device status word, one per device (a __device__ variable is instantiated
+// per device by the runtime).
+__device__ unsigned g_dev_status;
+
+}  // namespace
+
+unsigned *device_status_ptr() {
+    static std::mutex mu;
+    static unsigned *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dev_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned *>(p);
+    }
+    return ptrs[dev];
+}
+
+int sm_count() {
+    static std::mutex mu;
+    static int counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+}  // namespace ks
+
+using namespace ks;
+
+extern "C" {
+
+ks_status ks_matmul_variant(const void *X, const void *values, int64_t a, int64_t b, int64_t c,
+                            int64_t d, int64_t batch, void *Y, int dtype, int variant, void *stream) {
+    if (variant < KS_VARIANT_AUTO || variant > KS_VARIANT_TC)
+        return fail(KS_ERR_INVALID_ARG, "unknown variant %d", variant);
+    Problem p;
+    bool noop = false;
+    ks_status s = make_problem(X, values, a, b, c, d, batch, Y, dtype, stream, &p, &noop);
+    if (s != KS_OK || noop) return s;
+    return run(p, variant);
+}
+
+ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b, int64_t c, int64_t d,
+                    int64_t batch, void *Y, int dtype, void *stream) {
+    return ks_matmul_variant(X, values, a, b, c, d, batch, Y, dtype, KS_VARIANT_AUTO, stream);
+}
+
+ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch, int dtype, int *variant) {
+    if (!variant) return fail(KS_ERR_INVALID_ARG, "variant must be non-null");
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    int64_t in_f, out_f, nvals;
+    if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
+    // Assume 256-byte aligned buffers, as a fresh allocation has.
+    static const char dummy[16] __attribute__((aligned(256))) = {};
+    Problem p{dummy, dummy, (void *)(dummy + 0), a, b, c, d, std::max<int64_t>(batch, 1), dtype, nullptr};
+    Plan plan;
+    const char *why = "";
+    if (!make_plan(p, KS_VARIANT_AUTO, &plan, &why))
+        return fail(KS_ERR_UNSUPPORTED, "no kernel: %s", why);
+    *variant = plan.variant;
+    return KS_OK;
+}
+
+ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *patterns, int n_factors,
+                   int64_t batch, void *Y, int dtype, void *stream) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    if (n_factors <= 0 || !factors || !patterns)
+        return fail(KS_ERR_INVALID_ARG, "need n_factors > 0 and non-null factors/patterns");
+    int64_t widest = 0;
+    for (int t = 0; t < n_factors; ++t) {
+        const ks_pattern &q = patterns[t];
+        int64_t in_f, out_f, nvals;
+        if ((s = check_sizes(q.a, q.b, q.c, q.d, batch, &in_f, &out_f, &nvals)) != KS_OK) {
+            char tmp[512];
+            snprintf(tmp, sizeof(tmp), "factor %d: %s", t, g_msg);
+            return fail(s, "%s", tmp);
+        }
+        if (t > 0) {
+            const ks_pattern &r = patterns[t - 1];
+            if (r.a * r.b * r.d != in_f)
+                return fail(KS_ERR_INVALID_ARG, "factor %d has input width %lld but factor %d outputs %lld", t,
+                            (long long)in_f, t - 1, (long long)(r.a * r.b * r.d));
+        }
+        if (t < n_factors - 1) widest = std::max(widest, out_f);
+        if (!factors[t]) return fail(KS_ERR_INVALID_ARG, "factor %d is null", t);
+    }
+    if (batch == 0) return KS_OK;
+    if (!X || !Y) return fail(KS_ERR_INVALID_ARG, "X and Y must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_factors == 1) {
+        const ks_pattern &q = patterns[0];
+        return ks_matmul(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
+    }
+    // Two ping-pong intermediates, stream-ordered.
+    void *buf[2] = {nullptr, nullptr};
+    const size_t bytes = (size_t)batch * (size_t)widest * (size_t)elem;
+    for (int k = 0; k < 2 && k < n_factors - 1; ++k) {
+        cudaError_t e = cudaMallocAsync(&buf[k], bytes, st);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            if (buf[0]) (void)cudaFreeAsync(buf[0], st);
+            return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", bytes, cudaGetErrorString(e));
+        }
+    }
+    const void *src = X;
+    ks_status result = KS_OK;
+    for (int t = 0; t < n_factors; ++t) {
+        const ks_pattern &q = patterns[t];
+        void *dst = (t == n_factors - 1) ? Y : buf[t & 1];
+        result = ks_matmul(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, stream);
+        if (result != KS_OK) {
+            char tmp[512];
+            snprintf(tmp, sizeof(tmp), "factor %d: %s", t, g_msg);
+            fail(result, "%s", tmp);
+            break;
+        }
+        src = dst;
+    }
+    for (int k = 0; k < 2; ++k)
+        if (buf[k]) {
+            cudaError_t e = cudaFreeAsync(buf[k], st);
+            if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+        }
+    return result;
+}
+
+const char *ks_last_error(void) { return g_msg; }
+
+const char *ks_status_string(int status) {
+    switch (status) {
+        case KS_OK: return "KS_OK";
+        case KS_ERR_INVALID_ARG: return "KS_ERR_INVALID_ARG";
+        case KS_ERR_MISALIGNED: return "KS_ERR_MISALIGNED";
+        case KS_ERR_UNSUPPORTED: return "KS_ERR_UNSUPPORTED";
+        case KS_ERR_ALLOC: return "KS_ERR_ALLOC";
+        case KS_ERR_CUDA: return "KS_ERR_CUDA";
+        case KS_ERR_TIMEOUT: return "KS_ERR_TIMEOUT";
+        default: return "KS_ERR_UNKNOWN";
+    }
+}
+
+ks_status ks_sync_status(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned *p = device_status_ptr();
+    if (!p) return fail(KS_ERR_CUDA, "device status word unavailable");
+    unsigned v = 0;
+    e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading device status");
+    if (v != 0) {
+        unsigned zero = 0;
+        e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing device status");
+        if (v & kDevTimeout) return fail(KS_ERR_TIMEOUT, "a bounded device-side wait gave up (status 0x%x)", v);
+        return fail(KS_ERR_CUDA, "device status 0x%x", v);
+    }
+    return KS_OK;
+}
+
+int ks_version(void) { return 100; }
+
+}  // extern "C"

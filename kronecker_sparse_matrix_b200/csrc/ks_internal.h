@@ -1,0 +1,73 @@
+// Internal interfaces between the C ABI (ks_api.cu), the pattern heuristic
+// (ks_plan.cu) and the kernel families (ks_stream.cu, ks_fma.cu, ks_tc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ks.h"
+
+namespace ks {
+
+// One KS product, after validation: Y = X K^T with K of pattern (a,b,c,d).
+struct Problem {
+    const void *X;
+    const void *V;  // values[a][d][b][c]
+    void *Y;
+    int64_t a, b, c, d, batch;
+    int dtype;      // ks_dtype
+    cudaStream_t stream;
+
+    int64_t in_features() const { return a * c * d; }
+    int64_t out_features() const { return a * b * d; }
+    int elem_bytes() const { return dtype == KS_BF16 ? 2 : 4; }
+};
+
+// Tile choice of the CUDA-core gather-GEMM (see ks_fma.cu).
+struct FmaConfig {
+    int dl;  // l values per CTA (1, 2, 4 or 8)
+    int wm;  // warps along rows per l   (warp tile 64 rows)
+    int wk;  // warps along k per l      (warp tile 4*tn k)
+    int tn;  // k per thread (8, 12 or 16)
+};
+
+// Tile choice of the tcgen05 block-GEMM (see ks_tc.cu).
+struct TcConfig {
+    int dl;  // l values per CTA
+    int bk;  // k values per CTA tile (MMA N)
+    int ct;  // j values per pipeline stage
+};
+
+struct Plan {
+    int variant;  // ks_variant, never AUTO
+    FmaConfig fma;
+    TcConfig tc;
+};
+
+// Heuristic (ks_plan.cu).  Returns false if `variant` (possibly forced) cannot
+// run this problem; `why` then says so.
+bool make_plan(const Problem &p, int variant, Plan *out, const char **why);
+
+// Capability checks used by the heuristic.
+bool stream_supported(const Problem &p);
+bool fma_supported(const Problem &p, const char **why);
+bool tc_supported(const Problem &p, const char **why);
+FmaConfig fma_choose(const Problem &p);
+TcConfig tc_choose(const Problem &p);
+
+// Launchers: return cudaSuccess or the launch error.  Pure device work on
+// p.stream; no allocation, no synchronisation.
+cudaError_t launch_stream(const Problem &p);
+cudaError_t launch_fma(const Problem &p, const FmaConfig &cfg);
+cudaError_t launch_tc(const Problem &p, const TcConfig &cfg);
+
+// Device status word (ks_api.cu): kernels OR these bits in on failure.
+enum DeviceStatusBits : unsigned {
+    kDevTimeout = 1u,
+};
+unsigned *device_status_ptr();  // address of the status word on the current device
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace ks

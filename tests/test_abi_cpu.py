@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/ks.h declares, validates arguments on the host and plans kernels.
+No call here reaches a CUDA API (all of them fail validation first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kronecker_sparse_matrix_b200 import _lib, build as ksbuild
+from kronecker_sparse_matrix_b200 import plan
+from kronecker_sparse_matrix_b200.inputs import sweep_patterns, butterfly_patterns
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ks.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ksbuild.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(ks_[a-z_]+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for n in ["ks_matmul", "ks_matmul_variant", "ks_chain", "ks_plan", "ks_last_error",
+              "ks_status_string", "ks_sync_status", "ks_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding misses {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ks_version() >= 100
+    assert lib.ks_status_string(0) == b"KS_OK"
+    assert lib.ks_status_string(6) == b"KS_ERR_TIMEOUT"
+    assert lib.ks_status_string(99) == b"KS_ERR_UNKNOWN"
+
+
+P = 1 << 20  # a fake 256-byte-aligned address; never dereferenced (validation fails first)
+
+
+@pytest.mark.parametrize("pat", [(0, 1, 1, 1), (1, -2, 1, 1), (1, 1, 0, 1), (1, 1, 1, -1)])
+def test_bad_pattern_is_invalid(lib, pat):
+    assert lib.ks_matmul(P, P, *pat, 4, P * 8, 0, None) == 1
+    assert b"positive" in lib.ks_last_error()
+
+
+def test_negative_batch_bad_dtype_null_pointers(lib):
+    assert lib.ks_matmul(P, P, 2, 2, 2, 2, -1, P * 8, 0, None) == 1
+    assert lib.ks_matmul(P, P, 2, 2, 2, 2, 4, P * 8, 7, None) == 1
+    assert lib.ks_matmul(None, P, 2, 2, 2, 2, 4, P * 8, 0, None) == 1
+    assert lib.ks_matmul(P, P, 2, 2, 2, 2, 4, None, 0, None) == 1
+    assert lib.ks_matmul_variant(P, P, 2, 2, 2, 2, 4, P * 8, 0, 9, None) == 1
+
+
+def test_overflow_is_invalid(lib):
+    big = 1 << 40
+    assert lib.ks_matmul(P, P, big, big, 2, 2, 4, P * 8, 0, None) == 1
+    assert b"overflow" in lib.ks_last_error() or b"2^31" in lib.ks_last_error()
+
+
+def test_zero_batch_is_a_noop(lib):
+    assert lib.ks_matmul(None, None, 2, 2, 2, 2, 0, None, 0, None) == 0
+
+
+def test_misaligned_pointers(lib):
+    assert lib.ks_matmul(P + 2, P, 2, 2, 2, 2, 4, P * 8, 0, None) == 2   # fp32 needs 4 bytes
+    assert lib.ks_matmul(P, P, 2, 2, 2, 2, 4, P * 8 + 1, 2, None) == 2   # bf16 needs 2 bytes
+
+
+def test_overlapping_output_is_invalid(lib):
+    # Y = X: 4 rows of 8 fp32
+    assert lib.ks_matmul(P, P * 4, 2, 2, 2, 2, 4, P, 0, None) == 1
+    assert b"overlaps X" in lib.ks_last_error()
+    assert lib.ks_matmul(P, P * 4, 2, 2, 2, 2, 4, P * 4 + 16, 0, None) == 1
+    assert b"overlaps values" in lib.ks_last_error()
+
+
+def test_chain_validation(lib):
+    pats = (_lib.KsPattern * 2)(_lib.KsPattern(1, 2, 2, 2), _lib.KsPattern(1, 2, 2, 1))
+    ptrs = (ctypes.c_void_p * 2)(P, P)
+    assert lib.ks_chain(P, ptrs, pats, 2, 4, P * 8, 0, None) == 1
+    assert b"input width" in lib.ks_last_error()
+    assert lib.ks_chain(P, ptrs, pats, 0, 4, P * 8, 0, None) == 1
+    ok = (_lib.KsPattern * 2)(_lib.KsPattern(1, 2, 2, 2), _lib.KsPattern(2, 2, 2, 1))
+    null = (ctypes.c_void_p * 2)(P, None)
+    assert lib.ks_chain(P, null, ok, 2, 4, P * 8, 0, None) == 1
+    assert lib.ks_chain(P, ptrs, ok, 2, 0, P * 8, 0, None) == 0  # batch 0: no-op
+
+
+def test_plan_is_host_only_and_sensible(lib):
+    v = ctypes.c_int(-1)
+    assert lib.ks_plan(1, 192, 48, 8, 25216, 0, ctypes.byref(v)) == 0
+    assert v.value == _lib.KS_VARIANT_FMA
+    for p in butterfly_patterns(12):
+        assert plan(p, 4096) == "stream"
+    for p in sweep_patterns():
+        assert plan(p, 25088) == "fma"
+    assert plan((3, 5, 7, 3), 10) == "stream"  # odd d: the scalar catch-all
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load()
