@@ -1,0 +1,574 @@
+"""Benchmark: KS matmul throughput on B200 as a fraction of its roofline.
+
+Workload (default): the seeded sweep of 258 KS patterns
+(a, d in {1,...,64}; (b, c) in {(48,48),...,(256,256),(192,48),(256,64)};
+a*b*d, a*c*d <= 16384) at batch 25088, in fp32 and in bf16 -- 516 runs.  It
+stands in for the "600 KS patterns" of the KS-matmul abstract on the
+taxoreview.com page, whose list the pages do not give.  One step is one
+``ks_matmul`` launch per run (inputs resident in HBM, L2 flushed by a 256 MiB
+write before every timed launch, each launch timed alone by CUDA events on its
+stream).
+
+Per run r: FLOPs_r = 2*N*a*b*c*d, bytes_r = s*(N*a*c*d + N*a*b*d + a*b*c*d),
+roofline_r = min(P_peak, BW * FLOPs_r / bytes_r) with BW the measured HBM copy
+bandwidth, P_peak the fp32 FMA peak (148 SMs x 128 lanes x 2 x 1965 MHz) for
+fp32 runs and the measured bf16 tensor peak for bf16 runs;
+frac_r = (FLOPs_r / t_r) / roofline_r.  ``value`` is the median of frac_r over
+the runs.  One JSON line is printed (rank 0).
+
+``--impl reference`` times the CPU oracle (the plain C loops under oracle/)
+on a bounded sample of the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from kronecker_sparse_matrix_b200 import inputs  # noqa: E402
+
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12  # 74.45: SMs x FP32 lanes x 2 flop x max SM clock
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "KS matmul GFLOP/s and HBM GB/s at 1 B200 as fraction of roofline, pattern median"
+L2_FLUSH_BYTES = 256 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------- peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def run_flops(p, n):
+    a, b, c, d = p
+    return 2.0 * n * a * b * c * d
+
+
+def run_bytes(p, n, s):
+    a, b, c, d = p
+    return float(s) * (n * a * c * d + n * a * b * d + a * b * c * d)
+
+
+def roofline_tflops(p, n, dtype, peaks):
+    s = 4 if dtype == "fp32" else 2
+    ai = run_flops(p, n) / run_bytes(p, n, s)
+    p_peak = FP32_FMA_PEAK_TFLOPS if dtype in ("fp32", "tf32") else peaks["bf16_tflops"]
+    return min(p_peak, peaks["hbm_gbs"] * ai / 1e3)
+
+
+# ---------------------------------------------------------------------------- workloads
+def workload_runs(name):
+    """List of (label, pattern, batch, dtype, seed)."""
+    if name == "sweep":
+        pats = inputs.sweep_patterns()
+        return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16") for i, p in enumerate(pats)]
+    if name == "sweep-fp32":
+        return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "fp32", i) for i, p in enumerate(inputs.sweep_patterns())]
+    if name == "sweep-quick":  # every 8th pattern, for development only
+        pats = inputs.sweep_patterns()
+        return [(f"sweep[{i}]", pats[i], inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16")
+                for i in range(0, len(pats), 8)]
+    if name == "vit":
+        return [("vit", inputs.VIT_PATTERN, inputs.VIT_BATCH, "fp32", 0)]
+    if name == "gpt2":
+        return [("gpt2-fp32", inputs.GPT2_PATTERN, inputs.GPT2_BATCH, "fp32", 0),
+                ("gpt2-bf16", inputs.GPT2_PATTERN, inputs.GPT2_BATCH, "bf16", 0)]
+    raise ValueError(name)
+
+
+WORKLOAD_TEXT = {
+    "sweep": "seeded KS pattern sweep: 258 patterns x {fp32, bf16} = 516 runs, batch 25088 "
+             "(a,d in {1,2,4,...,64}; (b,c) in {(48,48),(64,64),(96,96),(128,128),(192,192),(256,256),"
+             "(192,48),(256,64)}; a*b*d, a*c*d <= 16384); X ~ N(0,1), values ~ N(0,1/c), seed = pattern index",
+}
+
+
+def torch_dtype(dt):
+    return torch.float32 if dt in ("fp32", "tf32") else torch.bfloat16
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (every 200 ms)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, path=None):
+        self.gpu_index = gpu_index
+        self.path = path
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self.path:
+                with open(self.path, "w") as f:
+                    f.write("\n".join(self.lines) + "\n")
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(values, world, device):
+    """Elementwise max over ranks of a list of floats (the per-run times)."""
+    if world <= 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def rank_seed(seed, rank):
+    """Weak scaling: rank r draws its own batch of rows (units are independent rows)."""
+    return seed + 1_000_003 * rank
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kronecker_sparse_matrix_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(variant_key):
+    """Per-launch DRAM traffic of the dominant kernel from a committed ncu
+    summary, or None when missing or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tr = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = tr.get(variant_key)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def gpu_arm(args, rank, world, local):
+    import kronecker_sparse_matrix_b200 as ks
+
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    runs = workload_runs(args.workload)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    results = []
+    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if args.save_clocks else None
+
+    # --- device-resident timing ------------------------------------------------
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local, clock_path) as clocks:
+        for label, p, n, dt, seed in runs:
+            f = inputs.factor_inputs(p, n, seed=rank_seed(seed, rank), dtype=torch_dtype(dt), device=dev)
+            Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
+            variant = ks.plan(p, n, ks.ks_dtype_of(f.X))
+            for _ in range(args.warmup):
+                ks.matmul(f.X, f.values, p, out=Y)
+            times = []
+            for _ in range(args.steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                ks.matmul(f.X, f.values, p, out=Y)
+                e1.record(stream)
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1) / 1e3)
+            results.append({"label": label, "pattern": p, "batch": n, "dtype": dt, "variant": variant,
+                            "times": times})
+            del f, Y
+        ks.sync_status()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+
+    # max over ranks, per run and step
+    flat = [t for r in results for t in r["times"]]
+    flat = max_over_ranks(flat, world, dev)
+    k = 0
+    for r in results:
+        r["times"] = flat[k:k + args.steps]
+        k += args.steps
+
+    for r in results:
+        p, n, dt = r["pattern"], r["batch"], r["dtype"]
+        t = statistics.mean(r["times"])
+        s = 4 if dt == "fp32" else 2
+        r["t"] = t
+        r["flops"] = run_flops(p, n) * world
+        r["bytes"] = run_bytes(p, n, s) * world
+        r["roof_tflops"] = roofline_tflops(p, n, dt, peaks) * world
+        r["tflops"] = r["flops"] / t / 1e12
+        r["frac"] = r["tflops"] / r["roof_tflops"]
+
+    # --- end to end through the public API with host buffers -------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_measure(args, runs, rank, world, dev, peaks)
+
+    return results, peaks, clocks.summary(), e2e
+
+
+def e2e_measure(args, runs, rank, world, dev, peaks):
+    """Same runs, each with H2D copies of X and values from pinned host memory,
+    the KS product, and the D2H copy of Y, all inside the timed region."""
+    import kronecker_sparse_matrix_b200 as ks
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    max_x = max(n * inputs.in_features(p) * (4 if dt == "fp32" else 2) for _, p, n, dt, _ in runs)
+    max_y = max(n * inputs.out_features(p) * (4 if dt == "fp32" else 2) for _, p, n, dt, _ in runs)
+    max_v = max(p[0] * p[1] * p[2] * p[3] * 4 for _, p, _, _, _ in runs)
+    hx = torch.empty(max_x, dtype=torch.uint8, pin_memory=True)
+    hy = torch.empty(max_y, dtype=torch.uint8, pin_memory=True)
+    hv = torch.empty(max_v, dtype=torch.uint8, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+    fracs = [[] for _ in runs]
+    h2d = d2h = 0
+    for ri, (label, p, n, dt, seed) in enumerate(runs):
+        f = inputs.factor_inputs(p, n, seed=rank_seed(seed, rank), dtype=torch_dtype(dt), device=dev)
+        es = f.X.element_size()
+        xb, vb = f.X.numel() * es, f.values.numel() * es
+        yb = n * inputs.out_features(p) * es
+        hxv = hx[:xb].view(f.X.dtype).view(f.X.shape)
+        hvv = hv[:vb].view(f.values.dtype).view(f.values.shape)
+        hyv = hy[:yb].view(f.X.dtype).view(n, inputs.out_features(p))
+        hxv.copy_(f.X)
+        hvv.copy_(f.values)
+        dX, dV = torch.empty_like(f.X), torch.empty_like(f.values)
+        dY = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
+        del f
+        # warm-up once (untimed)
+        dX.copy_(hxv, non_blocking=True)
+        dV.copy_(hvv, non_blocking=True)
+        ks.matmul(dX, dV, p, out=dY)
+        hyv.copy_(dY, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        for _ in range(steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dX.copy_(hxv, non_blocking=True)
+            dV.copy_(hvv, non_blocking=True)
+            ks.matmul(dX, dV, p, out=dY)
+            hyv.copy_(dY, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            t = e0.elapsed_time(e1) / 1e3
+            fracs[ri].append(t)
+        h2d += xb + vb
+        d2h += yb
+        del dX, dV, dY
+    flat = max_over_ranks([t for fr in fracs for t in fr], world, dev)
+    vals = []
+    k = 0
+    for (label, p, n, dt, seed), fr in zip(runs, fracs):
+        t = statistics.mean(flat[k:k + len(fr)])
+        k += len(fr)
+        vals.append(run_flops(p, n) / t / 1e12 / roofline_tflops(p, n, dt, peaks))
+    return {"value": statistics.median(vals), "unit": "fraction of roofline (median over runs)",
+            "h2d_bytes_per_step": int(h2d * world), "d2h_bytes_per_step": int(d2h * world),
+            "steps": steps, "note": "per run: pinned-host H2D of X and values, ks_matmul, D2H of Y"}
+
+
+# ---------------------------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(runs, rows, seed_offset=0):
+    """Time the CPU oracle on `rows` rows of every run; returns per-run seconds and flops."""
+    import oracle
+
+    oracle.build()
+    out = []
+    for label, p, n, dt, seed in runs:
+        f = inputs.factor_inputs(p, rows, seed=seed + seed_offset, dtype=torch_dtype(dt), device="cpu")
+        X = f.X.double().numpy()
+        V = f.values.double().numpy()
+        t0 = time.perf_counter()
+        oracle.matmul(X, V, p)
+        t = time.perf_counter() - t0
+        out.append((p, dt, t, run_flops(p, rows)))
+    return out, oracle.threads()
+
+
+def oracle_fracs(samples, peaks, batch_for_roofline):
+    fr = []
+    for (p, dt, t, fl), n in zip(samples, batch_for_roofline):
+        fr.append(fl / t / 1e12 / roofline_tflops(p, n, dt, peaks))
+    return fr
+
+
+def cpu_baseline(args, runs, peaks):
+    rows = args.cpu_rows
+    samples, cores = oracle_sample(runs, rows)
+    fr = oracle_fracs(samples, peaks, [n for _, _, n, _, _ in runs])
+    tot_t = sum(s[2] for s in samples)
+    tot_f = sum(s[3] for s in samples)
+    return {"value": statistics.median(fr), "unit": "fraction of roofline (median over runs)", "cores": cores,
+            "kind": "oracle", "gflops": tot_f / tot_t / 1e9, "seconds": tot_t,
+            "sample": f"{rows} rows of every run of the workload ({len(runs)} runs), oracle in fp64 on "
+                      f"{cores} host threads; per-run throughput divided by that run's B200 roofline"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    runs = workload_runs(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(runs[:4], 2)
+    t_steps, fr_steps = [], []
+    cores = 1
+    for step in range(args.steps):
+        samples, cores = oracle_sample(runs, args.ref_rows, seed_offset=step)
+        t_steps.append(sum(s[2] for s in samples))
+        fr_steps.append(oracle_fracs(samples, peaks, [n for _, _, n, _, _ in runs]))
+    per_run = [statistics.mean(x) for x in zip(*fr_steps)]
+    value = statistics.median(per_run)
+    line = {"impl": "reference", "metric": METRIC, "value": value,
+            "unit": "fraction of roofline (median over runs)", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(t_steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload),
+                       "sample_rows_per_run": args.ref_rows},
+            "cpu_baseline": {"value": value, "unit": "fraction of roofline (median over runs)", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{args.ref_rows} rows of every run per step, fp64 C loops"},
+            "e2e": {"value": value, "unit": "fraction of roofline (median over runs)",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+# ---------------------------------------------------------------------------- extra configs
+def extra_configs(args, dev, peaks):
+    """ViT / GPT-2 single factors and the butterfly chain, device-timed."""
+    import kronecker_sparse_matrix_b200 as ks
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(ts)
+
+    out = {}
+    for name, dt in [("vit", "fp32"), ("gpt2", "fp32"), ("gpt2", "bf16")]:
+        f = getattr(inputs, name)(dtype=torch_dtype(dt), device=dev)
+        p, n = f.pattern, f.batch
+        Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
+        t = timed(lambda: ks.matmul(f.X, f.values, p, out=Y), args.steps)
+        s = 4 if dt == "fp32" else 2
+        tf = run_flops(p, n) / t / 1e12
+        out[f"{name}-{dt}"] = {"pattern": list(p), "batch": n, "us": t * 1e6, "tflops": tf,
+                               "gbs": run_bytes(p, n, s) / t / 1e9,
+                               "frac": tf / roofline_tflops(p, n, dt, peaks),
+                               "variant": ks.plan(p, n, ks.ks_dtype_of(f.X))}
+    c = inputs.butterfly(device=dev)
+    Y = torch.empty_like(c.X)
+    t = timed(lambda: ks.chain(c.X, c.factors, c.patterns, out=Y), args.steps)
+    byts = sum(run_bytes(p, c.batch, 4) for p in c.patterns)
+    out["butterfly-chain-fp32"] = {"factors": len(c.patterns), "batch": c.batch, "us": t * 1e6,
+                                   "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peaks["hbm_gbs"],
+                                   "note": "12 launches, HBM round trip per factor"}
+    return out
+
+
+# ---------------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ks", "reference"], default="ks")
+    ap.add_argument("--workload", default="sweep")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=128)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--save-clocks", action="store_true")
+    ap.add_argument("--details", default=None, help="write per-run results as JSON here")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        # CPU only: rank 0 runs the oracle, the other ranks exit without work.
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = reference_arm(args, rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    rank, world, local = dist_setup(args)
+    try:
+
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device (the reference arm runs on CPU: --impl reference)")
+        dev = torch.device("cuda", local)
+        results, peaks, clocks, e2e = gpu_arm(args, rank, world, local)
+        extra = extra_configs(args, dev, peaks) if (rank == 0 and not args.no_extra) else None
+        if rank != 0:
+            return 0
+        fracs = [r["frac"] for r in results]
+        value = statistics.median(fracs)
+        per_dtype = {dt: statistics.median([r["frac"] for r in results if r["dtype"] == dt])
+                     for dt in sorted({r["dtype"] for r in results})}
+        ms_per_step = 1e3 * sum(r["t"] for r in results)
+        tot_f = sum(r["flops"] for r in results)
+        tot_b = sum(r["bytes"] for r in results)
+        tot_t = sum(r["t"] for r in results)
+        # dominant kernel: the (variant, dtype) family with the most device time
+        fam = {}
+        for r in results:
+            key = f"{r['variant']}-{r['dtype']}"
+            e = fam.setdefault(key, {"t": 0.0, "flops": 0.0, "bytes": 0.0, "n": 0})
+            e["t"] += r["t"]
+            e["flops"] += r["flops"]
+            e["bytes"] += r["bytes"]
+            e["n"] += 1
+        dom_key = max(fam, key=lambda k: fam[k]["t"])
+        dom = fam[dom_key]
+        if dom_key.startswith("fma-fp32"):
+            achieved = dom["flops"] / dom["t"] / 1e12
+            roof = {"bound": "alu", "achieved": achieved, "peak": FP32_FMA_PEAK_TFLOPS, "unit": "TFLOP/s",
+                    "frac": achieved / FP32_FMA_PEAK_TFLOPS,
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
+        elif dom_key.startswith("tc"):
+            achieved = dom["bytes"] / dom["t"] / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+        else:
+            achieved = dom["bytes"] / dom["t"] / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+        roof["kernel"] = dom_key
+        roof["launches"] = dom["n"]
+        roof["traffic"] = ncu_traffic(dom_key)
+        roof["note"] = ("achieved = algorithmic flops (or bytes) summed over that family's launches / summed "
+                        "CUDA-event launch time")
+        line = {
+            "metric": METRIC, "value": value, "unit": "fraction of roofline (median over runs)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32+bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "runs": len(results),
+                       "batch_per_gpu": results[0]["batch"], "l2": "flushed by a 256 MiB write before every timed launch",
+                       "parallelism": f"dp{world} (rows sharded, no collective)" if world > 1 else "single GPU"},
+            "median_frac_by_dtype": per_dtype,
+            "aggregate": {"tflops": tot_f / tot_t / 1e12, "gbs": tot_b / tot_t / 1e9},
+            "roofline": roof,
+            "cpu_baseline": cpu_baseline(args, workload_runs(args.workload), peaks) if world == 1 else None,
+            "e2e": e2e,
+            "gpu_launches": len(results) * args.steps,
+            "clocks": clocks,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                      "fp32_fma_tflops": FP32_FMA_PEAK_TFLOPS, "source": peaks["source"]},
+            "extra": extra,
+        }
+        if args.details:
+            with open(args.details, "w") as f:
+                json.dump({"results": [{k: v for k, v in r.items()} for r in results], "line": line}, f, indent=1)
+        print(json.dumps(line), flush=True)
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())
