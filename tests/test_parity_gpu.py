@@ -161,3 +161,22 @@ def test_full_size_sweep_patterns_sampled_rows(idx, dtype):
     rows = sampled_rows(f.batch, k=24)
     ref = oracle.matmul(f.X[rows].cpu(), f.values.cpu(), p)
     assert oracle.max_rel_err(Y[rows].cpu(), ref) <= TOL[dtype]
+
+
+TC_CASES = [(1, 64, 64, 1), (1, 48, 48, 1), (2, 64, 64, 2), (1, 256, 64, 16), (1, 96, 96, 4), (4, 128, 128, 1),
+            (1, 48, 48, 8), (2, 192, 48, 8), (1, 256, 256, 2), (1, 16, 16, 1), (3, 32, 16, 4), (2, 64, 64, 32)]
+
+
+@pytest.mark.parametrize("p", TC_CASES)
+@pytest.mark.parametrize("batch", [1, 67, 300])
+def test_tc_kernel_bf16(p, batch):
+    run_and_check(p, batch, dtype=torch.bfloat16, variant="tc")
+
+
+def test_tc_rejects_fp32_and_unsupported():
+    f = inputs.factor_inputs((1, 64, 64, 1), 8)
+    with pytest.raises(ks.KsError):
+        ks.matmul(f.X.to(DEV), f.values.to(DEV), (1, 64, 64, 1), variant="tc")
+    g = inputs.factor_inputs((1, 64, 40, 1), 8, dtype=torch.bfloat16)  # c not a multiple of 16
+    with pytest.raises(ks.KsError):
+        ks.matmul(g.X.to(DEV), g.values.to(DEV), (1, 64, 40, 1), variant="tc")
