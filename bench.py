@@ -83,10 +83,17 @@ def workload_runs(name):
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16") for i, p in enumerate(pats)]
     if name == "sweep-fp32":
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "fp32", i) for i, p in enumerate(inputs.sweep_patterns())]
+    if name == "sweep-bf16":
+        return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "bf16", i) for i, p in enumerate(inputs.sweep_patterns())]
     if name == "sweep-quick":  # every 8th pattern, for development only
         pats = inputs.sweep_patterns()
         return [(f"sweep[{i}]", pats[i], inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16")
                 for i in range(0, len(pats), 8)]
+    if name.startswith("pattern:"):  # pattern:a,b,c,d:dtype[:batch] -- one run, seed 0
+        parts = name.split(":")
+        pat = tuple(int(v) for v in parts[1].split(","))
+        batch = int(parts[3]) if len(parts) > 3 else inputs.SWEEP_BATCH
+        return [(name, pat, batch, parts[2], 0)]
     if name == "vit":
         return [("vit", inputs.VIT_PATTERN, inputs.VIT_BATCH, "fp32", 0)]
     if name == "gpt2":
