@@ -116,6 +116,28 @@ ks_status ks_chain(const void *X, const void *const *factors,
                    const ks_pattern *patterns, int n_factors, int64_t batch,
                    void *Y, int dtype, void *stream);
 
+/* ks_chain without any device allocation (the paper has no counterpart: this
+ * entry point serves callers that must not allocate).  Callers whose device
+ * memory is owned by another allocator, such as a framework's caching pool, or
+ * who run latency-critical loops where an allocation is not allowed, cannot
+ * let ks_chain allocate its intermediates.  This variant keeps them in one
+ * fixed array inside the library instead: 32 MiB per device, reserved on every
+ * GPU that loads the library and held until the process exits, split into two
+ * intermediates of at most 16 MiB each.
+ *
+ * Arguments, layouts and the result are exactly those of ks_chain.  A chain
+ * whose intermediate (batch x intermediate width x element size) exceeds
+ * 16 MiB is rejected with KS_ERR_INVALID_ARG before anything runs.  The
+ * first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call before
+ * any stream capture.  Nothing is cleared between calls: each intermediate is
+ * written in full before it is read.  All calls share the one array, so calls
+ * whose work overlaps on the GPU (other streams, other host threads) race on
+ * it: order them on one stream, or synchronise between them. */
+ks_status ks_chain_noalloc(const void *X, const void *const *factors,
+                           const ks_pattern *patterns, int n_factors,
+                           int64_t batch, void *Y, int dtype, void *stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char *ks_last_error(void);
 

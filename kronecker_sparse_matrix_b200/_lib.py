@@ -37,6 +37,7 @@ SIGNATURES = {
     "ks_matmul_variant": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp]),
     "ks_plan": (_int, [_i64, _i64, _i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "ks_chain": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
+    "ks_chain_noalloc": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
     "ks_last_error": (ctypes.c_char_p, []),
     "ks_status_string": (ctypes.c_char_p, [_int]),
     "ks_sync_status": (_int, [_vp]),

@@ -155,6 +155,14 @@ int sm_count() {
     return counts[dev];
 }
 
+ks_status record_error(ks_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
 }  // namespace ks
 
 using namespace ks;

@@ -70,4 +70,8 @@ unsigned *device_status_ptr();  // address of the status word on the current dev
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Records the message ks_last_error() returns on this host thread and passes
+// the status through (for entry points defined outside ks_api.cu).
+ks_status record_error(ks_status s, const char *fmt, ...);
+
 }  // namespace ks
