@@ -1,4 +1,5 @@
-// Output-stationary CUDA-core gather-GEMM for one KS factor.
+// Output-stationary CUDA-core gather-GEMM for one KS factor, register-staged
+// (bf16, and fp32 problems beyond the cp.async kernel's 32-bit tile index).
 //
 // Y[n, i*b*d + k*d + l] = sum_{j<c} values[i, l, k, j] * X[n, i*c*d + j*d + l]
 // (taxoreview.com page on Kronecker-sparse matrix multiplication, first
@@ -397,7 +398,12 @@ FmaConfig fma_choose(const Problem &p) {
 
 cudaError_t launch_fma(const Problem &p, const FmaConfig &c) {
     if (p.dtype == KS_BF16) return launch_typed<__nv_bfloat16>(p, c);
-    return launch_typed<float>(p, c);  // KS_F32, and KS_TF32 computed in full fp32
+    // fp32 (KS_F32, and KS_TF32 computed in full fp32) runs on the cp.async
+    // ring kernel; this register-staged one remains for grids whose tile count
+    // does not fit its 32-bit tile index.
+    const cudaError_t e = launch_fma32(p, c);
+    if (e != cudaErrorInvalidConfiguration) return e;
+    return launch_typed<float>(p, c);
 }
 
 }  // namespace ks

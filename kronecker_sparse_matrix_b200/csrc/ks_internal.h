@@ -59,6 +59,7 @@ TcConfig tc_choose(const Problem &p);
 // p.stream; no allocation, no synchronisation.
 cudaError_t launch_stream(const Problem &p);
 cudaError_t launch_fma(const Problem &p, const FmaConfig &cfg);
+cudaError_t launch_fma32(const Problem &p, const FmaConfig &cfg);  // fp32, cp.async ring (ks_fma32.cu)
 cudaError_t launch_tc(const Problem &p, const TcConfig &cfg);
 
 // Device status word (ks_api.cu): kernels OR these bits in on failure.
