@@ -108,10 +108,13 @@ ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
  * Widths must chain: a_t*b_t*d_t == a_{t+1}*c_{t+1}*d_{t+1}, else
  * KS_ERR_INVALID_ARG.  X is batch x (a_0*c_0*d_0), Y is
  * batch x (a_{n-1}*b_{n-1}*d_{n-1}).  Intermediates (in the chain's storage
- * dtype) live in two workspace buffers allocated stream-ordered
- * (cudaMallocAsync) and freed on the same stream before return
- * (KS_ERR_ALLOC if that fails).  Each factor runs the kernel the pattern
- * heuristic picks. */
+ * dtype) live in two workspace buffers allocated stream-ordered from a memory
+ * pool the library owns on each device (cudaMallocFromPoolAsync) and freed to
+ * it on the same stream before return (KS_ERR_ALLOC if the allocation fails).
+ * The pool keeps freed memory for later calls: the device memory it holds
+ * grows to the largest workspace one call has used and stays reserved until
+ * the process exits.  Each factor runs the kernel the pattern heuristic
+ * picks. */
 ks_status ks_chain(const void *X, const void *const *factors,
                    const ks_pattern *patterns, int n_factors, int64_t batch,
                    void *Y, int dtype, void *stream);

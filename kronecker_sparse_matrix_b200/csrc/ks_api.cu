@@ -141,6 +141,32 @@ unsigned *device_status_ptr() {
     return ptrs[dev];
 }
 
+// The chain workspace pool of the current device: a library-owned memory pool
+// whose release threshold keeps freed blocks for the next call (so a chain
+// call does not map and unmap its workspace every time), or nullptr.
+cudaMemPool_t chain_pool() {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            (void)cudaMemPoolDestroy(pool);
+            return nullptr;
+        }
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 int sm_count() {
     static std::mutex mu;
     static int counts[64] = {};
@@ -234,16 +260,25 @@ ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *
         const ks_pattern &q = patterns[0];
         return ks_matmul(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
     }
-    // Two ping-pong intermediates, stream-ordered.
+    // Two ping-pong intermediates in one stream-ordered allocation from the
+    // library's pool (256-byte aligned halves).
     void *buf[2] = {nullptr, nullptr};
-    const size_t bytes = (size_t)batch * (size_t)widest * (size_t)elem;
-    for (int k = 0; k < 2 && k < n_factors - 1; ++k) {
-        cudaError_t e = cudaMallocAsync(&buf[k], bytes, st);
+    const size_t bytes = ((size_t)batch * (size_t)widest * (size_t)elem + 255) / 256 * 256;
+    const size_t total = n_factors > 2 ? 2 * bytes : bytes;
+    cudaMemPool_t pool = chain_pool();
+    if (!pool) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
+    }
+    {
+        void *base = nullptr;
+        cudaError_t e = cudaMallocFromPoolAsync(&base, total, pool, st);
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
-            if (buf[0]) (void)cudaFreeAsync(buf[0], st);
-            return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", bytes, cudaGetErrorString(e));
+            return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", total, cudaGetErrorString(e));
         }
+        buf[0] = base;
+        if (n_factors > 2) buf[1] = static_cast<char *>(base) + bytes;
     }
     const void *src = X;
     ks_status result = KS_OK;
@@ -259,11 +294,10 @@ ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *
         }
         src = dst;
     }
-    for (int k = 0; k < 2; ++k)
-        if (buf[k]) {
-            cudaError_t e = cudaFreeAsync(buf[k], st);
-            if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
-        }
+    {
+        cudaError_t e = cudaFreeAsync(buf[0], st);
+        if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+    }
     return result;
 }
 

@@ -19,6 +19,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
+#include <cstdint>
 
 #include "ks_internal.h"
 
@@ -134,10 +136,195 @@ __global__ void __launch_bounds__(256) stream_scalar_kernel(const T *__restrict_
     }
 }
 
+// Blocks per unit of the merged layout: the least U with U*C*D and U*B*D
+// multiples of VEC (16-byte runs), or 0 if there is none up to VEC.
+__host__ __device__ constexpr int merged_units(int B, int C, int D, int VEC) {
+    for (int u = 1; u <= VEC; ++u)
+        if ((u * C * D) % VEC == 0 && (u * B * D) % VEC == 0) return u;
+    return 0;
+}
+
+// Register-weight streaming kernel for blocks of at most 4 x 4.  A thread owns
+// one "unit" of a row and keeps the unit's weights in registers while it walks
+// down a range of rows, so per row it moves only X in and Y out, as 16-byte
+// loads and stores:
+//   D == 0 (l-vector layout, d % VEC == 0): unit = (block i, VEC consecutive l);
+//          input j is the VEC-run at i*C*d + j*d + l0, output k the run at
+//          i*B*d + k*d + l0; weights values[i][l0 .. l0+VEC)[.][.] (contiguous);
+//   D == d (merged layout, d small): unit = U consecutive blocks, whose U*C*d
+//          inputs and U*B*d outputs are each one contiguous run; weights
+//          values[i0 .. i0+U)[.][.][.] (contiguous).
+// Threads form a TU x TR grid per CTA: TU consecutive units by TR row lanes.
+template <typename T, int B, int C, int D>
+__global__ void __launch_bounds__(256) stream_reg_kernel(const T *__restrict__ X, const T *__restrict__ V,
+                                                         T *__restrict__ Y, long long N, int d, int units,
+                                                         int in_f, int out_f, int tu_log2, int rows_per_cta) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int U = D == 0 ? 1 : merged_units(B, C, D, VEC);
+    static_assert(U > 0, "no 16-byte merged layout for this block shape");
+    constexpr int NL = D == 0 ? VEC : U * D;  // (block, l) lanes per unit
+    constexpr int NW = NL * B * C;            // weights per unit
+    const int tu = threadIdx.x & ((1 << tu_log2) - 1);
+    const int tr = threadIdx.x >> tu_log2;
+    const int TR = blockDim.x >> tu_log2;
+    const int u = (blockIdx.x << tu_log2) + tu;
+    if (u >= units) return;
+    const long long n_begin = (long long)blockIdx.y * rows_per_cta + tr;
+    const long long n_end = min(N, (long long)(blockIdx.y + 1) * rows_per_cta);
+
+    int x_off, y_off, w_off;
+    if constexpr (D == 0) {
+        const int dq = d / VEC;
+        const int i = u / dq, l0 = (u - i * dq) * VEC;
+        x_off = i * C * d + l0;
+        y_off = i * B * d + l0;
+        w_off = (i * d + l0) * B * C;
+    } else {
+        x_off = u * (U * C * D);
+        y_off = u * (U * B * D);
+        w_off = u * NW;
+    }
+    // w[q] = values at w_off + q: lane e, output k, input j at q = (e*B + k)*C + j
+    float w[NW];
+#pragma unroll
+    for (int q = 0; q < NW; q += VEC) {
+        float t[VEC];
+        Vec16<T>::load(V + w_off + q, t);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) w[q + e] = t[e];
+    }
+
+#pragma unroll 2
+    for (long long n = n_begin; n < n_end; n += TR) {
+        const T *x = X + n * in_f + x_off;
+        T *y = Y + n * out_f + y_off;
+        float xv[NL * C];  // xv[e*C + j]: lane e, input j
+        if constexpr (D == 0) {
+#pragma unroll
+            for (int j = 0; j < C; ++j) {
+                float t[VEC];
+                Vec16<T>::load(x + j * d, t);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) xv[e * C + j] = t[e];
+            }
+        } else {
+            // run layout [ub][j][l]; lane e = ub*D + l
+#pragma unroll
+            for (int q = 0; q < U * C * D; q += VEC) {
+                float t[VEC];
+                Vec16<T>::load(x + q, t);
+#pragma unroll
+                for (int r = 0; r < VEC; ++r) {
+                    const int f = q + r, ub = f / (C * D), j = (f / D) % C, l = f % D;
+                    xv[(ub * D + l) * C + j] = t[r];
+                }
+            }
+        }
+        float yv[NL * B];  // yv[e*B + k]
+#pragma unroll
+        for (int e = 0; e < NL; ++e)
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < C; ++j) acc = fmaf(w[(e * B + k) * C + j], xv[e * C + j], acc);
+                yv[e * B + k] = acc;
+            }
+        if constexpr (D == 0) {
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                float t[VEC];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) t[e] = yv[e * B + k];
+                Vec16<T>::store(y + k * d, t);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < U * B * D; q += VEC) {
+                float t[VEC];
+#pragma unroll
+                for (int r = 0; r < VEC; ++r) {
+                    const int f = q + r, ub = f / (B * D), k = (f / D) % B, l = f % D;
+                    t[r] = yv[(ub * D + l) * B + k];
+                }
+                Vec16<T>::store(y + q, t);
+            }
+        }
+    }
+}
+
 int grid_for(long long work, int threads) {
     long long blocks = (work + threads - 1) / threads;
     long long cap = (long long)sm_count() * 16;
     return (int)std::max<long long>(1, std::min(blocks, cap));
+}
+
+template <typename T, int B, int C, int D>
+cudaError_t launch_reg(const Problem &p) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int U = D == 0 ? 1 : merged_units(B, C, D, VEC);
+    const long long units = D == 0 ? p.a * p.d / VEC : p.a / U;
+    int tu_log2 = 0;
+    while ((1LL << tu_log2) < units && tu_log2 < 8) ++tu_log2;
+    const int TU = 1 << tu_log2, TR = 256 / TU;
+    const long long bx = (units + TU - 1) / TU;
+    const long long target = (long long)sm_count() * 8;  // 8 CTAs of 256 threads per SM
+    const long long max_by = std::min<long long>(65535, (p.batch + TR - 1) / TR);
+    const long long by = std::max<long long>(1, std::min(max_by, (target + bx - 1) / bx));
+    const long long rows_per_cta = (p.batch + by - 1) / by;
+    if (bx > INT32_MAX || rows_per_cta > INT32_MAX) return cudaErrorInvalidConfiguration;
+    stream_reg_kernel<T, B, C, D><<<dim3((unsigned)bx, (unsigned)by), 256, 0, p.stream>>>(
+        static_cast<const T *>(p.X), static_cast<const T *>(p.V), static_cast<T *>(p.Y), p.batch, (int)p.d,
+        (int)units, (int)p.in_features(), (int)p.out_features(), tu_log2, (int)rows_per_cta);
+    return cudaGetLastError();
+}
+
+// The register-weight kernel for (b, c) in {1, 2, 4}^2, if the layout allows:
+// 16-byte aligned X, values and Y; d % VEC == 0 (l-vector layout), or d < VEC
+// with a merged unit of U blocks dividing a.  cudaErrorNotSupported otherwise.
+template <typename T, int B, int C>
+cudaError_t launch_reg_bc(const Problem &p) {
+    constexpr int VEC = Vec16<T>::N;
+    if (p.d % VEC == 0) return launch_reg<T, B, C, 0>(p);
+    switch (p.d) {
+        case 1:
+            if (merged_units(B, C, 1, VEC) && p.a % merged_units(B, C, 1, VEC) == 0) return launch_reg<T, B, C, 1>(p);
+            break;
+        case 2:
+            if (merged_units(B, C, 2, VEC) && p.a % merged_units(B, C, 2, VEC) == 0) return launch_reg<T, B, C, 2>(p);
+            break;
+        case 4:
+            if constexpr (VEC == 8) {
+                if (merged_units(B, C, 4, VEC) && p.a % merged_units(B, C, 4, VEC) == 0)
+                    return launch_reg<T, B, C, 4>(p);
+            }
+            break;
+        default: break;
+    }
+    return cudaErrorNotSupported;
+}
+
+template <typename T, int B>
+cudaError_t launch_reg_b(const Problem &p) {
+    switch (p.c) {
+        case 1: return launch_reg_bc<T, B, 1>(p);
+        case 2: return launch_reg_bc<T, B, 2>(p);
+        case 4: return launch_reg_bc<T, B, 4>(p);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <typename T>
+cudaError_t launch_reg_any(const Problem &p) {
+    const uintptr_t al = reinterpret_cast<uintptr_t>(p.X) | reinterpret_cast<uintptr_t>(p.V) |
+                         reinterpret_cast<uintptr_t>(p.Y);
+    if (al % 16) return cudaErrorNotSupported;
+    switch (p.b) {
+        case 1: return launch_reg_b<T, 1>(p);
+        case 2: return launch_reg_b<T, 2>(p);
+        case 4: return launch_reg_b<T, 4>(p);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 template <typename T>
@@ -146,6 +333,8 @@ cudaError_t launch_typed(const Problem &p) {
     const T *X = static_cast<const T *>(p.X);
     const T *V = static_cast<const T *>(p.V);
     T *Y = static_cast<T *>(p.Y);
+    const cudaError_t er = launch_reg_any<T>(p);
+    if (er != cudaErrorNotSupported) return er;
     const bool aligned = (reinterpret_cast<uintptr_t>(p.X) % 16 == 0) && (reinterpret_cast<uintptr_t>(p.Y) % 16 == 0);
     if (aligned && p.d % VEC == 0) {
         const long long total = p.batch * p.a * (p.d / VEC);

@@ -73,6 +73,21 @@ def test_fma_kernel_bf16(p):
     run_and_check(p, 70, dtype=torch.bfloat16, variant="fma")
 
 
+# Block shapes (b, c) in {1, 2, 4}^2 take the register-weight streaming kernel:
+# d a multiple of the 16-byte element count (l-vector layout), or d in
+# {1, 2} (and 4 for bf16) with whole blocks merged into 16-byte runs; a
+# includes values the merged unit does not divide (those fall back).
+STREAM_REG = [(a, b, c, d) for (b, c) in [(1, 1), (1, 2), (2, 1), (2, 2), (2, 4), (4, 2), (4, 4), (1, 4)]
+              for (a, d) in [(8, 1), (4, 2), (2, 4), (2, 8), (3, 1), (1, 16), (6, 2)]]
+
+
+@pytest.mark.parametrize("p", STREAM_REG)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_stream_register_kernel_layouts(p, dtype):
+    for batch in (1, 7, 300):
+        run_and_check(p, batch, dtype=dtype, variant="stream")
+
+
 @pytest.mark.parametrize("p", [(2, 2, 2, 8), (4, 8, 8, 4), (1, 3, 3, 16), (2, 4, 4, 1)])
 def test_stream_kernel_bf16(p):
     run_and_check(p, 37, dtype=torch.bfloat16, variant="stream")
