@@ -114,10 +114,30 @@ ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
  * The pool keeps freed memory for later calls: the device memory it holds
  * grows to the largest workspace one call has used and stays reserved until
  * the process exits.  Each factor runs the kernel the pattern heuristic
- * picks. */
+ * picks, except for the chains ks_chain_ex fuses (see there). */
 ks_status ks_chain(const void *X, const void *const *factors,
                    const ks_pattern *patterns, int n_factors, int64_t batch,
                    void *Y, int dtype, void *stream);
+
+/* Flags of ks_chain_ex. */
+typedef enum ks_chain_flags {
+    KS_CHAIN_UNFUSED = 1 /* apply every factor with its own kernel, never a fused one */
+} ks_chain_flags;
+
+/* ks_chain with flags (a bitwise OR of ks_chain_flags; other bits:
+ * KS_ERR_INVALID_ARG).  ks_chain(...) is ks_chain_ex(..., 0, stream).
+ *
+ * Fusion: the twelve-factor 4096-wide butterfly chain, factors
+ * (2^t, 2, 2, 2^(11-t)) for t = 0..11 in that order (the square butterfly
+ * of size 4096, factor t mixing index bit 11 - t), runs as one kernel that
+ * reads X once and writes Y once, keeps intermediates in fp32 (also for bf16
+ * chains, which then round only Y) and allocates nothing.  It needs Y
+ * 16-byte aligned and the factors 16-byte (fp32) or 8-byte (bf16) aligned;
+ * otherwise, or with KS_CHAIN_UNFUSED, the chain runs factor by factor as
+ * described for ks_chain.  Y must not overlap X or a factor. */
+ks_status ks_chain_ex(const void *X, const void *const *factors,
+                      const ks_pattern *patterns, int n_factors, int64_t batch,
+                      void *Y, int dtype, int flags, void *stream);
 
 /* ks_chain without any device allocation (the paper has no counterpart: this
  * entry point serves callers that must not allocate).  Callers whose device

@@ -17,7 +17,7 @@ import torch
 
 from . import _lib
 from ._lib import (KS_BF16, KS_F32, KS_TF32, KS_VARIANT_AUTO, KS_VARIANT_FMA,  # noqa: F401
-                   KS_VARIANT_STREAM, KS_VARIANT_TC, KsError, KsPattern, VARIANTS)
+                   KS_CHAIN_UNFUSED, KS_VARIANT_STREAM, KS_VARIANT_TC, KsError, KsPattern, VARIANTS)
 
 Pattern = Tuple[int, int, int, int]
 
@@ -72,9 +72,10 @@ def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Opti
 
 
 def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[Pattern], *,
-          out: Optional[torch.Tensor] = None, tf32: bool = False,
+          out: Optional[torch.Tensor] = None, tf32: bool = False, fused: bool = True,
           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Y = X (K_{n-1} ... K_0)^T, factor 0 applied first."""
+    """Y = X (K_{n-1} ... K_0)^T, factor 0 applied first.  fused=False forces
+    one kernel per factor (ks_chain_ex with KS_CHAIN_UNFUSED)."""
     lib = _lib.load()
     n = len(factors)
     if n == 0 or len(patterns) != n:
@@ -92,7 +93,8 @@ def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[P
     ptrs = (ctypes.c_void_p * n)(*[f.data_ptr() for f in factors])
     pats = (KsPattern * n)(*[KsPattern(*[int(v) for v in p]) for p in patterns])
     with torch.cuda.device(x.device):
-        st = lib.ks_chain(x.data_ptr(), ptrs, pats, n, batch, out.data_ptr(), dt, _stream_ptr(stream, x.device))
+        st = lib.ks_chain_ex(x.data_ptr(), ptrs, pats, n, batch, out.data_ptr(), dt, 0 if fused else KS_CHAIN_UNFUSED,
+                             _stream_ptr(stream, x.device))
     _lib.check(st)
     return out
 

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "libks_b200.so")
 KS_F32, KS_TF32, KS_BF16 = 0, 1, 2
 # ks_variant
 KS_VARIANT_AUTO, KS_VARIANT_STREAM, KS_VARIANT_FMA, KS_VARIANT_TC = 0, 1, 2, 3
+KS_CHAIN_UNFUSED = 1
 VARIANTS = {"auto": 0, "stream": 1, "fma": 2, "tc": 3}
 # ks_status
 STATUS = {0: "KS_OK", 1: "KS_ERR_INVALID_ARG", 2: "KS_ERR_MISALIGNED", 3: "KS_ERR_UNSUPPORTED",
@@ -37,6 +38,7 @@ SIGNATURES = {
     "ks_matmul_variant": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp]),
     "ks_plan": (_int, [_i64, _i64, _i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "ks_chain": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
+    "ks_chain_ex": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp]),
     "ks_chain_noalloc": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
     "ks_last_error": (ctypes.c_char_p, []),
     "ks_status_string": (ctypes.c_char_p, [_int]),

@@ -230,6 +230,12 @@ ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch, int
 
 ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *patterns, int n_factors,
                    int64_t batch, void *Y, int dtype, void *stream) {
+    return ks_chain_ex(X, factors, patterns, n_factors, batch, Y, dtype, 0, stream);
+}
+
+ks_status ks_chain_ex(const void *X, const void *const *factors, const ks_pattern *patterns, int n_factors,
+                      int64_t batch, void *Y, int dtype, int flags, void *stream) {
+    if (flags & ~KS_CHAIN_UNFUSED) return fail(KS_ERR_INVALID_ARG, "unknown chain flags 0x%x", flags);
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
     if (n_factors <= 0 || !factors || !patterns)
@@ -259,6 +265,21 @@ ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *
     if (n_factors == 1) {
         const ks_pattern &q = patterns[0];
         return ks_matmul(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
+    }
+    if (!(flags & KS_CHAIN_UNFUSED) && butterfly12_matches(patterns, n_factors)) {
+        if ((s = check_align(X, elem, "X")) != KS_OK || (s = check_align(Y, elem, "Y")) != KS_OK) return s;
+        for (int t = 0; t < n_factors; ++t)
+            if ((s = check_align(factors[t], elem, "a factor")) != KS_OK) return s;
+        const int64_t width = 4096 * (int64_t)elem * batch;
+        if (ranges_overlap(Y, width, X, width)) return fail(KS_ERR_INVALID_ARG, "Y overlaps X");
+        for (int t = 0; t < n_factors; ++t)
+            if (ranges_overlap(Y, width, factors[t], 4096 * 2 * (int64_t)elem))
+                return fail(KS_ERR_INVALID_ARG, "Y overlaps factor %d", t);
+        if (butterfly12_supported(X, factors, Y, dtype)) {
+            const cudaError_t e = launch_butterfly12(X, factors, batch, Y, dtype, 8, st);
+            if (e != cudaSuccess) return cuda_fail(e, "fused butterfly chain launch");
+            return ok();
+        }
     }
     // Two ping-pong intermediates in one stream-ordered allocation from the
     // library's pool (256-byte aligned halves).

@@ -62,6 +62,13 @@ cudaError_t launch_fma(const Problem &p, const FmaConfig &cfg);
 cudaError_t launch_fma32(const Problem &p, const FmaConfig &cfg);  // fp32, cp.async ring (ks_fma32.cu)
 cudaError_t launch_tc(const Problem &p, const TcConfig &cfg);
 
+// Fused 4096-wide butterfly chain (ks_butterfly.cu): the twelve factors
+// (2^t, 2, 2, 2^(11-t)), t = 0..11, in that order.
+bool butterfly12_matches(const ks_pattern *patterns, int n);
+bool butterfly12_supported(const void *X, const void *const *factors, void *Y, int dtype);
+cudaError_t launch_butterfly12(const void *X, const void *const *factors, long long batch, void *Y, int dtype,
+                               int rows_per_block, cudaStream_t stream);
+
 // Device status word (ks_api.cu): kernels OR these bits in on failure.
 enum DeviceStatusBits : unsigned {
     kDevTimeout = 1u,

@@ -52,3 +52,48 @@ def test_chain_of_one_equals_matmul():
     f = inputs.factor_inputs((2, 64, 64, 2), 30)
     X, V = f.X.to(DEV), f.values.to(DEV)
     assert torch.equal(ks.chain(X, [V], [(2, 64, 64, 2)]), ks.matmul(X, V, (2, 64, 64, 2)))
+
+
+# The 4096-wide twelve-factor butterfly runs as one fused kernel (intermediates
+# in fp32): compare it with the oracle's chain, and with the factor-by-factor
+# path, on batches that leave a ragged last row block.
+@pytest.mark.parametrize("batch", [1, 5, 300])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fused_butterfly_matches_oracle(batch, dtype):
+    c = inputs.butterfly(device=DEV, dtype=dtype, batch=batch, seed=7)
+    Y = ks.chain(c.X, c.factors, c.patterns)
+    ks.sync_status()
+    ref = oracle.chain(c.X.cpu(), [f.cpu() for f in c.factors], c.patterns)
+    tol = 1e-5 if dtype == torch.float32 else 1e-2  # bf16: inputs exact, one output rounding
+    assert oracle.max_rel_err(Y.cpu(), ref) <= tol
+
+
+def test_fused_and_unfused_butterfly_agree():
+    c = inputs.butterfly(device=DEV, batch=64, seed=8)
+    fused = ks.chain(c.X, c.factors, c.patterns)
+    unfused = ks.chain(c.X, c.factors, c.patterns, fused=False)
+    ks.sync_status()
+    assert oracle.max_rel_err(fused.cpu(), unfused.cpu().double()) <= 1e-5
+
+
+def test_fused_butterfly_hadamard_is_exact():
+    pats = inputs.butterfly_patterns(12)
+    h2 = torch.tensor([[1.0, 1.0], [1.0, -1.0]])
+    facs = [h2.expand(p[0], p[3], 2, 2).contiguous().to(DEV) for p in pats]
+    rows = torch.tensor([0, 1, 5, 777, 4095])
+    X = torch.zeros(len(rows), 4096, device=DEV)
+    X[torch.arange(len(rows)), rows.to(DEV)] = 1.0
+    Y = ks.chain(X, facs, pats).cpu().numpy()
+    cols = np.arange(4096)
+    closed = np.array([[(-1.0) ** bin(int(r) & int(y)).count("1") for y in cols] for r in rows])
+    np.testing.assert_array_equal(Y, closed)
+
+
+def test_misaligned_output_falls_back_to_factor_kernels():
+    c = inputs.butterfly(device=DEV, batch=9, seed=9)
+    buf = torch.empty(9 * 4096 + 1, device=DEV)
+    out = buf[1:].view(9, 4096)  # 4-byte aligned, not 16
+    ks.chain(c.X, c.factors, c.patterns, out=out)
+    ks.sync_status()
+    ref = oracle.chain(c.X.cpu(), [f.cpu() for f in c.factors], c.patterns)
+    assert oracle.max_rel_err(out.cpu(), ref) <= 1e-5
