@@ -210,10 +210,21 @@ def rank_seed(seed, rank):
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def kernel_source_hash():
+# Source files of each kernel family: a recorded ncu traffic figure stays
+# valid only while these are unchanged.
+FAMILY_SOURCES = {
+    "fma-fp32": ["ks_fma32.cu", "ks_fma.cu", "ks_internal.h"],
+    "fma-bf16": ["ks_fma.cu", "ks_internal.h"],
+    "tc-bf16": ["ks_tc.cu", "ks_sm100.cuh", "ks_internal.h"],
+    "stream-fp32": ["ks_stream.cu", "ks_internal.h"],
+    "stream-bf16": ["ks_stream.cu", "ks_internal.h"],
+}
+
+
+def kernel_source_hash(family):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kronecker_sparse_matrix_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in FAMILY_SOURCES.get(family, sorted(os.listdir(csrc))):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -229,9 +240,9 @@ def ncu_traffic(variant_key):
     except (OSError, ValueError):
         return None
     ent = tr.get(variant_key)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(variant_key):
         return None
-    return ent.get("bytes_per_launch")
+    return ent
 
 
 def gpu_arm(args, rank, world, local):
@@ -461,13 +472,22 @@ def extra_configs(args, dev, peaks):
                                "gbs": run_bytes(p, n, s) / t / 1e9,
                                "frac": tf / roofline_tflops(p, n, dt, peaks),
                                "variant": ks.plan(p, n, ks.ks_dtype_of(f.X))}
-    c = inputs.butterfly(device=dev)
-    Y = torch.empty_like(c.X)
-    t = timed(lambda: ks.chain(c.X, c.factors, c.patterns, out=Y), args.steps)
-    byts = sum(run_bytes(p, c.batch, 4) for p in c.patterns)
-    out["butterfly-chain-fp32"] = {"factors": len(c.patterns), "batch": c.batch, "us": t * 1e6,
-                                   "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peaks["hbm_gbs"],
-                                   "note": "12 launches, HBM round trip per factor"}
+    for dt in ("fp32", "bf16"):
+        c = inputs.butterfly(device=dev, dtype=torch_dtype(dt))
+        s = 4 if dt == "fp32" else 2
+        Y = torch.empty_like(c.X)
+        vbytes = sum(p[0] * p[1] * p[2] * p[3] for p in c.patterns) * s
+        for fused in (True, False):
+            t = timed(lambda: ks.chain(c.X, c.factors, c.patterns, out=Y, fused=fused), args.steps)
+            if fused:  # X once, Y once, every factor's values once
+                byts = 2 * s * c.batch * c.X.shape[1] + vbytes
+                note = "one fused kernel: X read once, Y written once"
+            else:      # every factor's X and Y through HBM
+                byts = sum(run_bytes(p, c.batch, s) for p in c.patterns)
+                note = "12 launches, HBM round trip per factor"
+            out[f"butterfly-chain-{dt}" + ("" if fused else "-unfused")] = {
+                "factors": len(c.patterns), "batch": c.batch, "us": t * 1e6, "algorithmic_bytes": byts,
+                "gbs": byts / t / 1e9, "frac": byts / t / 1e9 / peaks["hbm_gbs"], "note": note}
     return out
 
 
@@ -543,7 +563,12 @@ def main(argv=None):
                     "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
         roof["kernel"] = dom_key
         roof["launches"] = dom["n"]
-        roof["traffic"] = ncu_traffic(dom_key)
+        tr = ncu_traffic(dom_key)
+        roof["traffic"] = tr["bytes_per_launch"] if tr else None
+        if tr:
+            roof["traffic_note"] = (f"ncu DRAM read+write per launch, mean over the family's {tr['launches']} sweep "
+                                    f"launches; algorithmic bytes per launch {tr['algorithmic_bytes_per_launch']:.4g} "
+                                    f"(profiles/traffic.json)")
         roof["note"] = ("achieved = algorithmic flops (or bytes) summed over that family's launches / summed "
                         "CUDA-event launch time")
         line = {
