@@ -65,6 +65,10 @@ def _load():
             lib.ks_ref_chain.argtypes = [_dp, ctypes.POINTER(_dp),
                                          ctypes.POINTER(_i64), ctypes.c_int, _i64, _dp]
             lib.ks_ref_chain.restype = ctypes.c_int
+            lib.ks_ref_dx.argtypes = [_dp, _dp, _i64, _i64, _i64, _i64, _i64, _dp]
+            lib.ks_ref_dx.restype = None
+            lib.ks_ref_dv.argtypes = [_dp, _dp, _i64, _i64, _i64, _i64, _i64, _dp]
+            lib.ks_ref_dv.restype = None
             lib.ks_ref_set_threads.argtypes = [ctypes.c_int]
             lib.ks_ref_set_threads.restype = None
             lib.ks_ref_get_threads.argtypes = []
@@ -113,6 +117,36 @@ def matmul(X, values, pattern) -> np.ndarray:
     if N:
         _load().ks_ref_matmul(_ptr(X), _ptr(V), a, b, c, d, N, _ptr(Y))
     return Y
+
+
+def dx(dY, values, pattern) -> np.ndarray:
+    """Input gradient of Y = X K^T: dX = dY K, (N, a*c*d) from dY (N, a*b*d)."""
+    a, b, c, d = _check_pattern(pattern)
+    G = _f64(dY)
+    V = _f64(values).reshape(-1)
+    if V.size != a * b * c * d:
+        raise ValueError("values must hold a*b*c*d entries")
+    G = G.reshape(-1, a * b * d) if G.size else G.reshape(0, a * b * d)
+    N = G.shape[0]
+    H = np.zeros((N, a * c * d), dtype=np.float64)
+    if N:
+        _load().ks_ref_dx(_ptr(G), _ptr(V), a, b, c, d, N, _ptr(H))
+    return H
+
+
+def dv(dY, X, pattern) -> np.ndarray:
+    """Values gradient of Y = X K^T: dV[i][l][k][j] = sum_n dY[n,(i,k,l)] X[n,(i,j,l)],
+    returned flat in the values layout [a][d][b][c]."""
+    a, b, c, d = _check_pattern(pattern)
+    G = _f64(dY)
+    X = _f64(X)
+    G = G.reshape(-1, a * b * d) if G.size else G.reshape(0, a * b * d)
+    X = X.reshape(-1, a * c * d) if X.size else X.reshape(0, a * c * d)
+    if G.shape[0] != X.shape[0]:
+        raise ValueError("dY and X need the same number of rows")
+    dV = np.zeros(a * b * c * d, dtype=np.float64)
+    _load().ks_ref_dv(_ptr(G), _ptr(X), a, b, c, d, G.shape[0], _ptr(dV))
+    return dV
 
 
 def densify(values, pattern) -> np.ndarray:

@@ -144,3 +144,60 @@ int ks_ref_chain(const double *X, const double *const *factors,
     free(buf[1]);
     return 0;
 }
+
+/* Backward of Y = X * K^T (the page's KSLinear layer is trained by gradient
+ * descent; these are the two gradients of that product, written from the
+ * definition of K above).
+ *
+ * Input gradient: dX = dY * K, i.e. for every n, i, j, l
+ *     dX[n][i*c*d + j*d + l] = sum_{k<b} values[i][l][k][j] * dY[n][i*b*d + k*d + l].
+ * dY is N x (a*b*d), dX is N x (a*c*d). */
+void ks_ref_dx(const double *dY, const double *values,
+               int64_t a, int64_t b, int64_t c, int64_t d,
+               int64_t N, double *dX)
+{
+    const int64_t in_f = a * c * d;
+    const int64_t out_f = a * b * d;
+    int nt = ks_ref_get_threads();
+    (void)nt;
+#pragma omp parallel for schedule(static) num_threads(nt)
+    for (int64_t n = 0; n < N; ++n) {
+        const double *g = dY + n * out_f;
+        double *h = dX + n * in_f;
+        for (int64_t i = 0; i < a; ++i)
+            for (int64_t j = 0; j < c; ++j)
+                for (int64_t l = 0; l < d; ++l) {
+                    double acc = 0.0;
+                    for (int64_t k = 0; k < b; ++k)
+                        acc += g[i * b * d + k * d + l] *
+                               values[(i * d + l) * b * c + k * c + j];
+                    h[i * c * d + j * d + l] = acc;
+                }
+    }
+}
+
+/* Gradient of the values: for every i, l, k, j
+ *     dV[i][l][k][j] = sum_{n<N} dY[n][i*b*d + k*d + l] * X[n][i*c*d + j*d + l],
+ * the entries of dY^T * X at K's support, in the values layout [a][d][b][c].
+ * The sum over n runs in order n = 0..N-1. */
+void ks_ref_dv(const double *dY, const double *X,
+               int64_t a, int64_t b, int64_t c, int64_t d,
+               int64_t N, double *dV)
+{
+    const int64_t in_f = a * c * d;
+    const int64_t out_f = a * b * d;
+    int nt = ks_ref_get_threads();
+    (void)nt;
+#pragma omp parallel for schedule(static) num_threads(nt)
+    for (int64_t il = 0; il < a * d; ++il) {
+        const int64_t i = il / d, l = il % d;
+        for (int64_t k = 0; k < b; ++k)
+            for (int64_t j = 0; j < c; ++j) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n)
+                    acc += dY[n * out_f + i * b * d + k * d + l] *
+                           X[n * in_f + i * c * d + j * d + l];
+                dV[((i * d + l) * b + k) * c + j] = acc;
+            }
+    }
+}
