@@ -472,6 +472,20 @@ def extra_configs(args, dev, peaks):
                                "gbs": run_bytes(p, n, s) / t / 1e9,
                                "frac": tf / roofline_tflops(p, n, dt, peaks),
                                "variant": ks.plan(p, n, ks.ks_dtype_of(f.X))}
+    # KSLinear backward: dX = dY K (pattern (a, c, b, d), transposed blocks) and
+    # dV (reduction over the batch); same flops and bytes as the forward product
+    for name, dt in [("vit", "fp32"), ("gpt2", "fp32"), ("gpt2", "bf16")]:
+        f = getattr(inputs, name)(dtype=torch_dtype(dt), device=dev)
+        p, n = f.pattern, f.batch
+        g = torch.Generator(device=dev).manual_seed(1)
+        dy = torch.randn(n, inputs.out_features(p), generator=g, device=dev).to(f.X.dtype)
+        roof = roofline_tflops(p, n, dt, peaks)
+        for grad, fn in (("dx", lambda: ks.matmul_dx(dy, f.values, p)), ("dv", lambda: ks.matmul_dv(dy, f.X, p))):
+            t = timed(fn, args.steps)
+            tf = run_flops(p, n) / t / 1e12
+            out[f"{name}-{dt}-{grad}"] = {"pattern": list(p), "batch": n, "us": t * 1e6, "tflops": tf,
+                                          "frac": tf / roof}
+        del f, dy
     for dt in ("fp32", "bf16"):
         c = inputs.butterfly(device=dev, dtype=torch_dtype(dt))
         s = 4 if dt == "fp32" else 2

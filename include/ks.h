@@ -96,6 +96,32 @@ ks_status ks_matmul_variant(const void *X, const void *values, int64_t a,
                             int64_t b, int64_t c, int64_t d, int64_t batch,
                             void *Y, int dtype, int variant, void *stream);
 
+/* Input gradient of Y = X * K^T (training the page's KSLinear layer):
+ *     dX = dY * K,  dX[n][i*c*d + j*d + l] = sum_{k<b} values[i][l][k][j] * dY[n][i*b*d + k*d + l].
+ * dY is batch x (a*b*d), dX is batch x (a*c*d), values as for ks_matmul; all
+ * DEVICE pointers of one dtype.  dX is overwritten and must not overlap dY or
+ * values (KS_ERR_INVALID_ARG).  This is the KS product of pattern (a, c, b, d)
+ * with every block transposed: the library transposes the values into a
+ * stream-ordered workspace from its pool (a*b*c*d elements, freed before
+ * return; KS_ERR_ALLOC if that fails) and runs the kernel ks_matmul picks for
+ * (a, c, b, d).  batch == 0 is a no-op. */
+ks_status ks_matmul_dx(const void *dY, const void *values, int64_t a, int64_t b,
+                       int64_t c, int64_t d, int64_t batch, void *dX, int dtype,
+                       void *stream);
+
+/* Values gradient of Y = X * K^T:
+ *     dV[i][l][k][j] = sum_{n<batch} dY[n][i*b*d + k*d + l] * X[n][i*c*d + j*d + l],
+ * written (not accumulated) in the values layout [a][d][b][c].  dY is
+ * batch x (a*b*d), X batch x (a*c*d); DEVICE pointers of one dtype, dV must
+ * not overlap dY or X.  Sums are fp32: each CTA sums a range of rows in row
+ * order, and the partial sums of the ranges (a stream-ordered fp32 workspace
+ * from the library's pool, at most 256 MiB) are added in range order, so the
+ * result is deterministic; bf16 dV is rounded once at the end.  batch == 0
+ * writes zeros. */
+ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b,
+                       int64_t c, int64_t d, int64_t batch, void *dV, int dtype,
+                       void *stream);
+
 /* What KS_VARIANT_AUTO would run for this problem, written to *variant
  * (a ks_variant).  Host-only: touches no device. */
 ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,

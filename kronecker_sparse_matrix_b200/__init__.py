@@ -71,6 +71,84 @@ def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Opti
     return out
 
 
+def _check_pair(u: torch.Tensor, v: torch.Tensor, names: str) -> None:
+    if u.dim() != 2 or not u.is_cuda or not u.is_contiguous() or not v.is_contiguous():
+        raise ValueError(f"{names} must be contiguous CUDA tensors, the first 2-D")
+    if v.dtype != u.dtype or v.device != u.device:
+        raise ValueError(f"{names} must share dtype and device")
+
+
+def matmul_dx(dy: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Optional[torch.Tensor] = None,
+              tf32: bool = False, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Input gradient of Y = X K^T: dX = dY K, (batch, a*c*d) from dY (batch, a*b*d)."""
+    a, b, c, d = (int(v) for v in pattern)
+    _check_pair(dy, values, "dy and values")
+    if out is None:
+        out = torch.empty((dy.shape[0], a * c * d), dtype=dy.dtype, device=dy.device)
+    with torch.cuda.device(dy.device):
+        st = _lib.load().ks_matmul_dx(dy.data_ptr(), values.data_ptr(), a, b, c, d, dy.shape[0], out.data_ptr(),
+                                      ks_dtype_of(dy, tf32), _stream_ptr(stream, dy.device))
+    _lib.check(st)
+    return out
+
+
+def matmul_dv(dy: torch.Tensor, x: torch.Tensor, pattern: Pattern, *, out: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Values gradient of Y = X K^T: dV[i][l][k][j] = sum_n dY[n,(i,k,l)] X[n,(i,j,l)],
+    a tensor of shape (a, d, b, c) (fp32 sums; bf16 rounded once)."""
+    a, b, c, d = (int(v) for v in pattern)
+    _check_pair(dy, x, "dy and x")
+    if x.shape[0] != dy.shape[0]:
+        raise ValueError("dy and x need the same number of rows")
+    if out is None:
+        out = torch.empty((a, d, b, c), dtype=dy.dtype, device=dy.device)
+    with torch.cuda.device(dy.device):
+        st = _lib.load().ks_matmul_dv(dy.data_ptr(), x.data_ptr(), a, b, c, d, dy.shape[0], out.data_ptr(),
+                                      ks_dtype_of(dy), _stream_ptr(stream, dy.device))
+    _lib.check(st)
+    return out
+
+
+class _KSLinearFn(torch.autograd.Function):
+    """Y = X K^T with K the KS factor of `pattern`; both gradients on the GPU."""
+
+    @staticmethod
+    def forward(ctx, x, values, pattern):
+        ctx.pattern = pattern
+        ctx.save_for_backward(x, values)
+        return matmul(x, values.contiguous(), pattern)
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, values = ctx.saved_tensors
+        dy = dy.contiguous()
+        dx = matmul_dx(dy, values.contiguous(), ctx.pattern) if ctx.needs_input_grad[0] else None
+        dv = matmul_dv(dy, x, ctx.pattern).view(values.shape) if ctx.needs_input_grad[1] else None
+        return dx, dv, None
+
+
+class KSLinear(torch.nn.Module):
+    """A linear layer whose weight is one KS factor of pattern (a, b, c, d):
+    in_features a*c*d, out_features a*b*d, y = x K^T (+ bias).  The values are
+    a parameter of shape (a, d, b, c), drawn N(0, 1/c) (unit-variance outputs
+    for unit-variance inputs).  Leading dimensions of x are flattened."""
+
+    def __init__(self, pattern: Pattern, bias: bool = False, dtype=torch.float32, device=None):
+        super().__init__()
+        a, b, c, d = (int(v) for v in pattern)
+        self.pattern = (a, b, c, d)
+        self.in_features, self.out_features = a * c * d, a * b * d
+        self.values = torch.nn.Parameter(torch.randn(a, d, b, c, dtype=dtype, device=device) * (1.0 / c) ** 0.5)
+        self.bias = torch.nn.Parameter(torch.zeros(a * b * d, dtype=dtype, device=device)) if bias else None
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        y = _KSLinearFn.apply(x.reshape(-1, self.in_features).contiguous(), self.values, self.pattern)
+        if self.bias is not None:
+            y = y + self.bias
+        return y.reshape(*lead, self.out_features)
+
+
 def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[Pattern], *,
           out: Optional[torch.Tensor] = None, tf32: bool = False, fused: bool = True,
           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:

@@ -322,6 +322,94 @@ ks_status ks_chain_ex(const void *X, const void *const *factors, const ks_patter
     return result;
 }
 
+ks_status ks_matmul_dx(const void *dY, const void *values, int64_t a, int64_t b, int64_t c, int64_t d,
+                       int64_t batch, void *dX, int dtype, void *stream) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    int64_t in_f, out_f, nvals;
+    if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
+    if (batch == 0) return KS_OK;
+    if (!dY || !values || !dX) return fail(KS_ERR_INVALID_ARG, "dY, values and dX must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    if ((s = check_align(dY, elem, "dY")) != KS_OK || (s = check_align(values, elem, "values")) != KS_OK ||
+        (s = check_align(dX, elem, "dX")) != KS_OK)
+        return s;
+    if (ranges_overlap(dX, batch * in_f * elem, dY, batch * out_f * elem))
+        return fail(KS_ERR_INVALID_ARG, "dX overlaps dY");
+    if (ranges_overlap(dX, batch * in_f * elem, values, nvals * elem))
+        return fail(KS_ERR_INVALID_ARG, "dX overlaps values");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaMemPool_t pool = chain_pool();
+    if (!pool) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
+    }
+    void *vt = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&vt, (size_t)(nvals * elem), pool, st);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace allocation of %lld bytes failed: %s", (long long)(nvals * elem),
+                    cudaGetErrorString(e));
+    }
+    // dX = dY K is the KS product of pattern (a, c, b, d) with the blocks transposed.
+    ks_status result = KS_OK;
+    e = launch_transpose_blocks(values, vt, a * d, b, c, dtype, st);
+    if (e != cudaSuccess) result = cuda_fail(e, "values transpose launch");
+    if (result == KS_OK) {
+        result = ks_matmul(dY, vt, a, c, b, d, batch, dX, dtype, stream);
+        if (result != KS_OK) {
+            char tmp[512];
+            snprintf(tmp, sizeof(tmp), "dX product: %s", g_msg);
+            fail(result, "%s", tmp);
+        }
+    }
+    e = cudaFreeAsync(vt, st);
+    if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+    return result;
+}
+
+ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
+                       void *dV, int dtype, void *stream) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    int64_t in_f, out_f, nvals;
+    if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
+    if (!dV) return fail(KS_ERR_INVALID_ARG, "dV must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    if ((s = check_align(dV, elem, "dV")) != KS_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (batch == 0) {  // an empty sum
+        cudaError_t e = cudaMemsetAsync(dV, 0, (size_t)(nvals * elem), st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "dV clear");
+    }
+    if (!dY || !X) return fail(KS_ERR_INVALID_ARG, "dY and X must be non-null");
+    if ((s = check_align(dY, elem, "dY")) != KS_OK || (s = check_align(X, elem, "X")) != KS_OK) return s;
+    if (ranges_overlap(dV, nvals * elem, dY, batch * out_f * elem)) return fail(KS_ERR_INVALID_ARG, "dV overlaps dY");
+    if (ranges_overlap(dV, nvals * elem, X, batch * in_f * elem)) return fail(KS_ERR_INVALID_ARG, "dV overlaps X");
+    DvProblem q{dY, X, dV, a, b, c, d, batch, dtype, st};
+    int splits = 1;
+    long long rows_per_split = batch;
+    dv_split(q, &splits, &rows_per_split);
+    cudaMemPool_t pool = chain_pool();
+    if (!pool) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
+    }
+    const size_t wbytes = (size_t)splits * (size_t)nvals * sizeof(float);
+    void *w = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&w, wbytes, pool, st);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", wbytes, cudaGetErrorString(e));
+    }
+    ks_status result = KS_OK;
+    e = launch_dv(q, static_cast<float *>(w), splits, rows_per_split);
+    if (e != cudaSuccess) result = cuda_fail(e, "dV kernel launch");
+    e = cudaFreeAsync(w, st);
+    if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+    return result == KS_OK ? ok() : result;
+}
+
 const char *ks_last_error(void) { return g_msg; }
 
 const char *ks_status_string(int status) {

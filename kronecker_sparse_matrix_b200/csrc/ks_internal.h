@@ -62,6 +62,25 @@ cudaError_t launch_fma(const Problem &p, const FmaConfig &cfg);
 cudaError_t launch_fma32(const Problem &p, const FmaConfig &cfg);  // fp32, cp.async ring (ks_fma32.cu)
 cudaError_t launch_tc(const Problem &p, const TcConfig &cfg);
 
+// Gradients (ks_backward.cu).  dV[i][l][k][j] = sum_n dY[n,(i,k,l)] X[n,(i,j,l)]
+// is computed over `splits` row ranges into fp32 partials W[split][a][d][b][c],
+// then reduced into dV (dtype of dY/X).
+struct DvProblem {
+    const void *dY, *X;
+    void *dV;
+    int64_t a, b, c, d, batch;
+    int dtype;
+    cudaStream_t stream;
+};
+int dv_dl(int64_t d);
+void dv_split(const DvProblem &q, int *splits, long long *rows_per_split);
+cudaError_t launch_dv(const DvProblem &q, float *W, int splits, long long rows_per_split);
+// vt[blk][j][k] = v[blk][k][j] for `blocks` blocks of b x c (KS values transposed per (i, l)).
+cudaError_t launch_transpose_blocks(const void *v, void *vt, int64_t blocks, int64_t b, int64_t c, int dtype,
+                                    cudaStream_t stream);
+// The library's retaining workspace pool of the current device (ks_api.cu).
+cudaMemPool_t chain_pool();
+
 // Fused 4096-wide butterfly chain (ks_butterfly.cu): the twelve factors
 // (2^t, 2, 2, 2^(11-t)), t = 0..11, in that order.
 bool butterfly12_matches(const ks_pattern *patterns, int n);
