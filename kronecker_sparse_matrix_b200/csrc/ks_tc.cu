@@ -13,7 +13,9 @@
 // 0, else DLS = d).  Its outputs for all l and all k of a pass (DLS * bp <=
 // 512 fp32 columns) accumulate in tensor memory while X streams through a
 // ring of 16/32 KB chunks exactly once per pass; most patterns need a single
-// pass, so X is read once and Y written once.
+// pass, so X is read once and Y written once.  Each pass is its own tile, and
+// the passes of one X tile are consecutive tiles, which run at the same time on
+// neighbouring CTAs and share X through L2.
 //
 //   warp 0      TMA producer: raw X chunks (128 rows x 64..128 (j, l)
 //               elements; l innermost, the only shape a tensor map can fetch
@@ -136,11 +138,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t xq = 0, vq = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-                const int g = (int)(tile % p.n_g);
-                const long long rb = tile / p.n_g;
+                const int ps = (int)(tile % p.passes);
+                const long long t2 = tile / p.passes;
+                const int g = (int)(t2 % p.n_g);
+                const long long rb = t2 / p.n_g;
                 const int i = g / groups_per_i, l0 = (g % groups_per_i) * DLS;
                 const int n0 = (int)(rb * kRows);
-                for (int ps = 0; ps < p.passes && ok; ++ps) {
+                {
                     for (int ch = 0; ch < n_chunks && ok; ++ch) {
                         const int xs = xq % S;
                         ok = mbar_wait(&x_empty[xs], ((xq / S) & 1) ^ 1, abort_flag, p.status);
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t xq = 0, vq = 0, accq = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-                for (int ps = 0; ps < p.passes && ok; ++ps, ++accq) {
+                for (int once = 0; once < 1 && ok; ++once, ++accq) {
                     const int buf = (int)(accq % p.nbuf);
                     ok = mbar_wait(&acc_empty[buf], ((accq / p.nbuf) & 1) ^ 1, abort_flag, p.status);
                     if (!ok) break;
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t xq = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-                for (int ps = 0; ps < p.passes && ok; ++ps) {
+                {
                     for (int ch = 0; ch < n_chunks; ++ch, ++xq) {
                         const int xs = xq % S;
                         const bool w = mbar_wait(&x_full[xs], (xq / S) & 1, abort_flag, p.status);
@@ -288,11 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t accq = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-            const int g = (int)(tile % p.n_g);
-            const long long rb = tile / p.n_g;
+            const int ps = (int)(tile % p.passes);
+            const long long t2 = tile / p.passes;
+            const int g = (int)(t2 % p.n_g);
+            const long long rb = t2 / p.n_g;
             const int i = g / groups_per_i, l0 = (g % groups_per_i) * DLS;
             const int row0 = (int)(rb * kRows) + 32 * quad;
-            for (int ps = 0; ps < p.passes && ok; ++ps, ++accq) {
+            for (int once = 0; once < 1 && ok; ++once, ++accq) {
                 const int buf = (int)(accq % p.nbuf);
                 ok = mbar_wait(&acc_full[buf], (accq / p.nbuf) & 1, abort_flag, p.status);
                 ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
@@ -410,7 +416,10 @@ int tc_kc(int dls, int bp) {
     return 0;
 }
 
-// k per pass: the largest multiple of 16 dividing b with dls * bp <= 512 and bp <= 256.
+// k per pass: the largest multiple of 16 dividing b with dls * bp <= 512 and
+// bp <= 256 (a single accumulator buffer when dls * bp > 256; smaller passes
+// that fit twice were measured slower: every extra pass repeats the transpose
+// of each X chunk).
 int tc_bp(int dls, int64_t b) {
     for (int bp = std::min(256, 512 / dls); bp >= 16; bp -= 16)
         if (b % bp == 0) return bp;
@@ -529,7 +538,10 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.kc = kc;
     p.nbuf = (2 * DLS * bp <= 512) ? 2 : 1;
     if (p.kc == 0) return cudaErrorInvalidConfiguration;
-    p.n_tiles = ((pr.batch + kRows - 1) / kRows) * p.n_g;
+    // tiles = (row block, l group, pass of k), the pass varying fastest: CTAs
+    // that run side by side take the passes of the same X tile, so its second
+    // read is served by L2
+    p.n_tiles = ((pr.batch + kRows - 1) / kRows) * p.n_g * p.passes;
     p.Y = static_cast<__nv_bfloat16 *>(pr.Y);
     p.status = device_status_ptr();
     if (!p.status) return cudaErrorUnknown;
