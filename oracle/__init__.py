@@ -22,6 +22,7 @@ products, the Sylvester-Hadamard closed form, hand-worked fixtures).
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 import threading
@@ -193,6 +194,39 @@ def chain(X, factors, patterns) -> np.ndarray:
             raise ValueError("chain widths do not match (a*b*d of factor t must equal "
                              "a*c*d of factor t+1)")
     return Y
+
+
+ACTIVATIONS = ("none", "relu", "gelu_tanh", "gelu_erf")
+
+
+def activation(Z, act: str) -> np.ndarray:
+    """The pointwise activations of the MLP shapes, on fp64 values, from their
+    definitions: relu(z) = max(z, 0); gelu_erf(z) = z * Phi(z) with
+    Phi(z) = (1 + erf(z / sqrt 2)) / 2; gelu_tanh(z) = z (1 + tanh(sqrt(2/pi)
+    (z + 0.044715 z^3))) / 2, the usual tanh form of the same function."""
+    Z = _f64(Z)
+    if act == "none":
+        return Z.copy()
+    if act == "relu":
+        return np.maximum(Z, 0.0)
+    if act == "gelu_erf":
+        erf = np.vectorize(math.erf, otypes=[np.float64])
+        return 0.5 * Z * (1.0 + erf(Z / math.sqrt(2.0)))
+    if act == "gelu_tanh":
+        return 0.5 * Z * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (Z + 0.044715 * Z ** 3)))
+    raise ValueError(f"unknown activation {act!r}")
+
+
+def matmul_epilogue(X, values, pattern, bias=None, act: str = "none") -> np.ndarray:
+    """act(X K^T + bias): the product, plus bias[col] on every row (bias has
+    a*b*d entries, or None), then the activation, all in fp64."""
+    Y = matmul(X, values, pattern)
+    if bias is not None:
+        B = _f64(bias).reshape(-1)
+        if B.size != Y.shape[1]:
+            raise ValueError("bias must hold a*b*d entries")
+        Y = Y + B[None, :]
+    return activation(Y, act)
 
 
 def max_rel_err(Y, Y_ref) -> float:
