@@ -472,6 +472,18 @@ def extra_configs(args, dev, peaks):
                                "gbs": run_bytes(p, n, s) / t / 1e9,
                                "frac": tf / roofline_tflops(p, n, dt, peaks),
                                "variant": ks.plan(p, n, ks.ks_dtype_of(f.X))}
+    # fused epilogue: act(X K^T + bias) with GELU (tanh form), the MLP-up layer
+    for name, dt in [("vit", "fp32"), ("gpt2", "bf16")]:
+        f = getattr(inputs, name)(dtype=torch_dtype(dt), device=dev)
+        p, n = f.pattern, f.batch
+        bias = torch.randn(inputs.out_features(p), generator=torch.Generator(device=dev).manual_seed(2),
+                           device=dev).to(f.X.dtype)
+        Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
+        t = timed(lambda: ks.matmul(f.X, f.values, p, out=Y, bias=bias, act="gelu_tanh"), args.steps)
+        tf = run_flops(p, n) / t / 1e12
+        out[f"{name}-{dt}-bias-gelu"] = {"pattern": list(p), "batch": n, "us": t * 1e6, "tflops": tf,
+                                         "frac": tf / roofline_tflops(p, n, dt, peaks)}
+        del f, Y
     # KSLinear backward: dX = dY K (pattern (a, c, b, d), transposed blocks) and
     # dV (reduction over the batch); same flops and bytes as the forward product
     for name, dt in [("vit", "fp32"), ("gpt2", "fp32"), ("gpt2", "bf16")]:

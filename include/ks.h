@@ -77,6 +77,17 @@ typedef enum ks_variant {
     KS_VARIANT_TC = 3      /* tcgen05 tensor-core block-GEMM (TF32 / BF16)     */
 } ks_variant;
 
+/* Pointwise activation of a fused epilogue (ks_matmul_ep, ks_chain_ep).
+ * GELU is z * Phi(z), Phi the standard normal distribution function, either
+ * exactly through erf or in the usual tanh form
+ * z * (1 + tanh(sqrt(2/pi) * (z + 0.044715 z^3))) / 2. */
+typedef enum ks_activation {
+    KS_ACT_NONE = 0,
+    KS_ACT_RELU = 1,      /* max(z, 0)                        */
+    KS_ACT_GELU_TANH = 2, /* GELU, tanh form (CUDA tanhf)     */
+    KS_ACT_GELU_ERF = 3   /* GELU, erf form (CUDA erff)       */
+} ks_activation;
+
 /* One factor's pattern: K is (a*b*d) x (a*c*d) with support I_a (x) 1_{b x c} (x) I_d. */
 typedef struct ks_pattern {
     int64_t a, b, c, d;
@@ -88,6 +99,19 @@ typedef struct ks_pattern {
 ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
                     int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
                     void *stream);
+
+/* ks_matmul with a fused epilogue (the MLP shapes' bias and activation):
+ *     Y[n][col] = act(sum_j ... + bias[col]),  col = i*b*d + k*d + l,
+ * computed on the fp32 accumulator before the single rounding to the storage
+ * dtype, inside the same kernel (no extra pass over Y).  bias is a DEVICE
+ * array of a*b*d elements of the storage dtype, or NULL for none; activation
+ * is a ks_activation (other values: KS_ERR_INVALID_ARG).  bias must not
+ * overlap Y.  variant is a ks_variant as for ks_matmul_variant.  With bias
+ * NULL, KS_ACT_NONE and KS_VARIANT_AUTO this is ks_matmul. */
+ks_status ks_matmul_ep(const void *X, const void *values, int64_t a, int64_t b,
+                       int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
+                       const void *bias, int activation, int variant,
+                       void *stream);
 
 /* ks_matmul with the kernel family forced (a ks_variant).  Returns
  * KS_ERR_UNSUPPORTED if that family cannot run this pattern / dtype /
@@ -164,6 +188,16 @@ typedef enum ks_chain_flags {
 ks_status ks_chain_ex(const void *X, const void *const *factors,
                       const ks_pattern *patterns, int n_factors, int64_t batch,
                       void *Y, int dtype, int flags, void *stream);
+
+/* ks_chain_ex with a fused epilogue on the last factor: Y = act(X (K_{n-1}
+ * ... K_0)^T + bias), bias of a_{n-1}*b_{n-1}*d_{n-1} elements or NULL (as in
+ * ks_matmul_ep).  A Monarch-style layer (two KS factors, then bias and
+ * activation) is one call.  With an epilogue the butterfly chain is not
+ * fused; its factors run one by one, the last with the epilogue. */
+ks_status ks_chain_ep(const void *X, const void *const *factors,
+                      const ks_pattern *patterns, int n_factors, int64_t batch,
+                      void *Y, int dtype, int flags, const void *bias,
+                      int activation, void *stream);
 
 /* ks_chain without any device allocation (the paper has no counterpart: this
  * entry point serves callers that must not allocate).  Callers whose device

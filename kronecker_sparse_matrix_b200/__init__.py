@@ -46,9 +46,12 @@ def _variant(v) -> int:
 
 
 def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Optional[torch.Tensor] = None,
-           tf32: bool = False, variant="auto", stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Y = X K^T for one KS factor.  x: (batch, a*c*d) CUDA tensor (fp32 or
-    bf16), values: a*b*c*d entries in [a][d][b][c] order, same dtype/device.
+           tf32: bool = False, variant="auto", bias: Optional[torch.Tensor] = None, act: str = "none",
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Y = act(X K^T + bias) for one KS factor.  x: (batch, a*c*d) CUDA tensor
+    (fp32 or bf16), values: a*b*c*d entries in [a][d][b][c] order, same
+    dtype/device; bias: a*b*d entries or None; act: "none", "relu",
+    "gelu_tanh" or "gelu_erf" (fused into the kernel's epilogue).
     Asynchronous on ``stream`` (default: the current stream)."""
     a, b, c, d = (int(v) for v in pattern)
     lib = _lib.load()
@@ -64,11 +67,26 @@ def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Opti
         out = torch.empty((batch, a * b * d), dtype=x.dtype, device=x.device)
     elif not out.is_contiguous() or out.dtype != x.dtype or out.device != x.device:
         raise ValueError("out must be contiguous with x's dtype and device")
+    bias_ptr = _bias_ptr(bias, x, a * b * d)
     with torch.cuda.device(x.device):
-        st = lib.ks_matmul_variant(x.data_ptr(), values.data_ptr(), a, b, c, d, batch, out.data_ptr(), dt,
-                                   _variant(variant), _stream_ptr(stream, x.device))
+        st = lib.ks_matmul_ep(x.data_ptr(), values.data_ptr(), a, b, c, d, batch, out.data_ptr(), dt, bias_ptr,
+                              _act(act), _variant(variant), _stream_ptr(stream, x.device))
     _lib.check(st)
     return out
+
+
+def _act(act: str) -> int:
+    if act not in _lib.ACTIVATIONS:
+        raise ValueError(f"act must be one of {sorted(_lib.ACTIVATIONS)}")
+    return _lib.ACTIVATIONS[act]
+
+
+def _bias_ptr(bias: Optional[torch.Tensor], x: torch.Tensor, n: int):
+    if bias is None:
+        return None
+    if bias.dtype != x.dtype or bias.device != x.device or not bias.is_contiguous() or bias.numel() != n:
+        raise ValueError(f"bias must be a contiguous tensor of {n} elements with x's dtype and device")
+    return bias.data_ptr()
 
 
 def _check_pair(u: torch.Tensor, v: torch.Tensor, names: str) -> None:
@@ -113,10 +131,10 @@ class _KSLinearFn(torch.autograd.Function):
     """Y = X K^T with K the KS factor of `pattern`; both gradients on the GPU."""
 
     @staticmethod
-    def forward(ctx, x, values, pattern):
+    def forward(ctx, x, values, bias, pattern):
         ctx.pattern = pattern
         ctx.save_for_backward(x, values)
-        return matmul(x, values.contiguous(), pattern)
+        return matmul(x, values.contiguous(), pattern, bias=bias)  # bias fused into the epilogue
 
     @staticmethod
     def backward(ctx, dy):
@@ -124,12 +142,14 @@ class _KSLinearFn(torch.autograd.Function):
         dy = dy.contiguous()
         dx = matmul_dx(dy, values.contiguous(), ctx.pattern) if ctx.needs_input_grad[0] else None
         dv = matmul_dv(dy, x, ctx.pattern).view(values.shape) if ctx.needs_input_grad[1] else None
-        return dx, dv, None
+        db = dy.sum(0) if ctx.needs_input_grad[2] else None
+        return dx, dv, db, None
 
 
 class KSLinear(torch.nn.Module):
     """A linear layer whose weight is one KS factor of pattern (a, b, c, d):
-    in_features a*c*d, out_features a*b*d, y = x K^T (+ bias).  The values are
+    in_features a*c*d, out_features a*b*d, y = x K^T (+ bias, fused into the
+    product's epilogue; its gradient is the column sum of dY).  The values are
     a parameter of shape (a, d, b, c), drawn N(0, 1/c) (unit-variance outputs
     for unit-variance inputs).  Leading dimensions of x are flattened."""
 
@@ -143,17 +163,18 @@ class KSLinear(torch.nn.Module):
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         lead = x.shape[:-1]
-        y = _KSLinearFn.apply(x.reshape(-1, self.in_features).contiguous(), self.values, self.pattern)
-        if self.bias is not None:
-            y = y + self.bias
+        y = _KSLinearFn.apply(x.reshape(-1, self.in_features).contiguous(), self.values, self.bias, self.pattern)
         return y.reshape(*lead, self.out_features)
 
 
 def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[Pattern], *,
           out: Optional[torch.Tensor] = None, tf32: bool = False, fused: bool = True,
+          bias: Optional[torch.Tensor] = None, act: str = "none",
           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """Y = X (K_{n-1} ... K_0)^T, factor 0 applied first.  fused=False forces
-    one kernel per factor (ks_chain_ex with KS_CHAIN_UNFUSED)."""
+    """Y = act(X (K_{n-1} ... K_0)^T + bias), factor 0 applied first, the
+    epilogue fused into the last factor's kernel.  fused=False forces one
+    kernel per factor (KS_CHAIN_UNFUSED).  Two factors with bias and GELU are
+    a Monarch-style MLP layer."""
     lib = _lib.load()
     n = len(factors)
     if n == 0 or len(patterns) != n:
@@ -171,8 +192,8 @@ def chain(x: torch.Tensor, factors: Sequence[torch.Tensor], patterns: Sequence[P
     ptrs = (ctypes.c_void_p * n)(*[f.data_ptr() for f in factors])
     pats = (KsPattern * n)(*[KsPattern(*[int(v) for v in p]) for p in patterns])
     with torch.cuda.device(x.device):
-        st = lib.ks_chain_ex(x.data_ptr(), ptrs, pats, n, batch, out.data_ptr(), dt, 0 if fused else KS_CHAIN_UNFUSED,
-                             _stream_ptr(stream, x.device))
+        st = lib.ks_chain_ep(x.data_ptr(), ptrs, pats, n, batch, out.data_ptr(), dt, 0 if fused else KS_CHAIN_UNFUSED,
+                             _bias_ptr(bias, x, a * b * d), _act(act), _stream_ptr(stream, x.device))
     _lib.check(st)
     return out
 

@@ -18,6 +18,7 @@ KS_F32, KS_TF32, KS_BF16 = 0, 1, 2
 # ks_variant
 KS_VARIANT_AUTO, KS_VARIANT_STREAM, KS_VARIANT_FMA, KS_VARIANT_TC = 0, 1, 2, 3
 KS_CHAIN_UNFUSED = 1
+ACTIVATIONS = {"none": 0, "relu": 1, "gelu_tanh": 2, "gelu_erf": 3}
 VARIANTS = {"auto": 0, "stream": 1, "fma": 2, "tc": 3}
 # ks_status
 STATUS = {0: "KS_OK", 1: "KS_ERR_INVALID_ARG", 2: "KS_ERR_MISALIGNED", 3: "KS_ERR_UNSUPPORTED",
@@ -38,6 +39,9 @@ SIGNATURES = {
     "ks_matmul_variant": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp]),
     "ks_plan": (_int, [_i64, _i64, _i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "ks_chain": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
+    "ks_matmul_ep": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp, _int, _int, _vp]),
+    "ks_chain_ep": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp,
+                           _int, _vp]),
     "ks_matmul_dx": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_matmul_dv": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_chain_ex": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp]),

@@ -211,6 +211,28 @@ ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b, int
     return ks_matmul_variant(X, values, a, b, c, d, batch, Y, dtype, KS_VARIANT_AUTO, stream);
 }
 
+ks_status ks_matmul_ep(const void *X, const void *values, int64_t a, int64_t b, int64_t c, int64_t d,
+                       int64_t batch, void *Y, int dtype, const void *bias, int activation, int variant,
+                       void *stream) {
+    if (variant < KS_VARIANT_AUTO || variant > KS_VARIANT_TC)
+        return fail(KS_ERR_INVALID_ARG, "unknown variant %d", variant);
+    if (activation < KS_ACT_NONE || activation > KS_ACT_GELU_ERF)
+        return fail(KS_ERR_INVALID_ARG, "unknown activation %d", activation);
+    Problem p;
+    bool noop = false;
+    ks_status s = make_problem(X, values, a, b, c, d, batch, Y, dtype, stream, &p, &noop);
+    if (s != KS_OK || noop) return s;
+    if (bias) {
+        const int elem = p.elem_bytes();
+        if ((s = check_align(bias, elem, "bias")) != KS_OK) return s;
+        if (ranges_overlap(Y, batch * p.out_features() * elem, bias, p.out_features() * elem))
+            return fail(KS_ERR_INVALID_ARG, "Y overlaps bias");
+    }
+    p.bias = bias;
+    p.act = activation;
+    return run(p, variant);
+}
+
 ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch, int dtype, int *variant) {
     if (!variant) return fail(KS_ERR_INVALID_ARG, "variant must be non-null");
     ks_status s = check_dtype(dtype);
@@ -235,7 +257,16 @@ ks_status ks_chain(const void *X, const void *const *factors, const ks_pattern *
 
 ks_status ks_chain_ex(const void *X, const void *const *factors, const ks_pattern *patterns, int n_factors,
                       int64_t batch, void *Y, int dtype, int flags, void *stream) {
+    return ks_chain_ep(X, factors, patterns, n_factors, batch, Y, dtype, flags, nullptr, KS_ACT_NONE, stream);
+}
+
+ks_status ks_chain_ep(const void *X, const void *const *factors, const ks_pattern *patterns, int n_factors,
+                      int64_t batch, void *Y, int dtype, int flags, const void *bias, int activation,
+                      void *stream) {
     if (flags & ~KS_CHAIN_UNFUSED) return fail(KS_ERR_INVALID_ARG, "unknown chain flags 0x%x", flags);
+    if (activation < KS_ACT_NONE || activation > KS_ACT_GELU_ERF)
+        return fail(KS_ERR_INVALID_ARG, "unknown activation %d", activation);
+    const bool has_ep = bias != nullptr || activation != KS_ACT_NONE;
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
     if (n_factors <= 0 || !factors || !patterns)
@@ -264,9 +295,9 @@ ks_status ks_chain_ex(const void *X, const void *const *factors, const ks_patter
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (n_factors == 1) {
         const ks_pattern &q = patterns[0];
-        return ks_matmul(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
+        return ks_matmul_ep(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, bias, activation, KS_VARIANT_AUTO, stream);
     }
-    if (!(flags & KS_CHAIN_UNFUSED) && butterfly12_matches(patterns, n_factors)) {
+    if (!(flags & KS_CHAIN_UNFUSED) && !has_ep && butterfly12_matches(patterns, n_factors)) {
         if ((s = check_align(X, elem, "X")) != KS_OK || (s = check_align(Y, elem, "Y")) != KS_OK) return s;
         for (int t = 0; t < n_factors; ++t)
             if ((s = check_align(factors[t], elem, "a factor")) != KS_OK) return s;
@@ -306,7 +337,10 @@ ks_status ks_chain_ex(const void *X, const void *const *factors, const ks_patter
     for (int t = 0; t < n_factors; ++t) {
         const ks_pattern &q = patterns[t];
         void *dst = (t == n_factors - 1) ? Y : buf[t & 1];
-        result = ks_matmul(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, stream);
+        result = (t == n_factors - 1)
+                     ? ks_matmul_ep(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, bias, activation,
+                                    KS_VARIANT_AUTO, stream)
+                     : ks_matmul(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, stream);
         if (result != KS_OK) {
             char tmp[512];
             snprintf(tmp, sizeof(tmp), "factor %d: %s", t, g_msg);

@@ -32,6 +32,7 @@
 #include <algorithm>
 #include <cstdint>
 
+#include "ks_epilogue.cuh"
 #include "ks_internal.h"
 
 namespace ks {
@@ -45,6 +46,8 @@ struct FmaParams {
     const void *X;
     const void *V;
     void *Y;
+    const void *bias;  // fused epilogue: out_f values of T, or null
+    int act;
     long long N;
     int a, b, c, d;
     int in_f, out_f;
@@ -281,8 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1) fma_kernel(const FmaParams p) {
                         const int fe = f + e;
                         v[e] = Cs[rr * TL::RS + (fe % DL) * TL::BKP + fe / DL];
                     }
-                    T *dst = Y + row * p.out_f + (long long)i * p.b * p.d + (long long)(k0 + kl) * p.d + l0 + ll;
-                    *reinterpret_cast<uint4 *>(dst) = Elem<T>::pack(v);
+                    const long long col = (long long)i * p.b * p.d + (long long)(k0 + kl) * p.d + l0 + ll;
+                    if (p.bias) {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) v[e] += ep_bias(static_cast<const T *>(p.bias), col + e);
+                    }
+                    if (p.act) ep_act_array(v, p.act);
+                    *reinterpret_cast<uint4 *>(Y + row * p.out_f + col) = Elem<T>::pack(v);
                 }
             }
             __syncthreads();
@@ -297,6 +305,8 @@ cudaError_t launch_cfg(const Problem &pr) {
     p.X = pr.X;
     p.V = pr.V;
     p.Y = pr.Y;
+    p.bias = pr.bias;
+    p.act = pr.act;
     p.N = pr.batch;
     p.a = (int)pr.a; p.b = (int)pr.b; p.c = (int)pr.c; p.d = (int)pr.d;
     p.in_f = (int)pr.in_features();

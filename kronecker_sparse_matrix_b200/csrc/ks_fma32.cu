@@ -28,6 +28,7 @@
 #include <climits>
 #include <cstdint>
 
+#include "ks_epilogue.cuh"
 #include "ks_internal.h"
 
 namespace ks {
@@ -41,6 +42,8 @@ struct Fma32Params {
     const float *X;
     const float *V;
     float *Y;
+    const float *bias;  // fused epilogue: out_f values or null
+    int act;
     long long N;
     int a, b, c, d;
     int bc;  // b * c
@@ -309,9 +312,13 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
                         const int fe = f + e;
                         v[e] = sEpi[rr * TL::RS + (fe % DL) * TL::BKP + fe / DL];
                     }
-                    float *out =
-                        p.Y + row * p.out_f + (long long)i * p.b * p.d + (long long)(k0 + kl) * p.d + l0 + ll;
-                    *reinterpret_cast<float4 *>(out) = make_float4(v[0], v[1], v[2], v[3]);
+                    const long long col = (long long)i * p.b * p.d + (long long)(k0 + kl) * p.d + l0 + ll;
+                    if (p.bias) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[e] += ep_bias(p.bias, col + e);
+                    }
+                    if (p.act) ep_act_array(v, p.act);
+                    *reinterpret_cast<float4 *>(p.Y + row * p.out_f + col) = make_float4(v[0], v[1], v[2], v[3]);
                 }
             }
             __syncthreads();
@@ -327,6 +334,8 @@ cudaError_t launch_cfg32(const Problem &pr) {
     p.X = static_cast<const float *>(pr.X);
     p.V = static_cast<const float *>(pr.V);
     p.Y = static_cast<float *>(pr.Y);
+    p.bias = static_cast<const float *>(pr.bias);
+    p.act = pr.act;
     p.N = pr.batch;
     p.a = (int)pr.a; p.b = (int)pr.b; p.c = (int)pr.c; p.d = (int)pr.d;
     p.bc = (int)(pr.b * pr.c);

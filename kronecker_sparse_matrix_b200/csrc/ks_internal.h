@@ -17,6 +17,10 @@ struct Problem {
     int64_t a, b, c, d, batch;
     int dtype;      // ks_dtype
     cudaStream_t stream;
+    // Fused epilogue Y = act(X K^T + bias): bias holds out_features() elements
+    // of the storage dtype (or is null), act is a ks_activation.
+    const void *bias = nullptr;
+    int act = 0;
 
     int64_t in_features() const { return a * c * d; }
     int64_t out_features() const { return a * b * d; }

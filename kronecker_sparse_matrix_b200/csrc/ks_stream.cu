@@ -22,6 +22,7 @@
 #include <climits>
 #include <cstdint>
 
+#include "ks_epilogue.cuh"
 #include "ks_internal.h"
 
 namespace ks {
@@ -70,7 +71,7 @@ __device__ __forceinline__ void from_f(__nv_bfloat16 &o, float v) { o = __float2
 template <typename T, int KB>
 __global__ void __launch_bounds__(256) stream_vec_kernel(const T *__restrict__ X, const T *__restrict__ V,
                                                          T *__restrict__ Y, long long total, int a, int b,
-                                                         int c, int d) {
+                                                         int c, int d, const T *__restrict__ bias, int act) {
     constexpr int VEC = Vec16<T>::N;
     const int dq = d / VEC;
     const long long in_f = (long long)a * c * d, out_f = (long long)a * b * d;
@@ -107,7 +108,15 @@ __global__ void __launch_bounds__(256) stream_vec_kernel(const T *__restrict__ X
 #pragma unroll
             for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
-                if (k < b) Vec16<T>::store(y + (long long)k * d, acc[kk]);
+                if (k < b) {
+                    if (bias) {
+                        const long long col = (long long)i * b * d + (long long)k * d + l0;
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) acc[kk][e] += ep_bias(bias, col + e);
+                    }
+                    if (act) ep_act_array(acc[kk], act);
+                    Vec16<T>::store(y + (long long)k * d, acc[kk]);
+                }
             }
         }
     }
@@ -117,7 +126,7 @@ __global__ void __launch_bounds__(256) stream_vec_kernel(const T *__restrict__ X
 template <typename T>
 __global__ void __launch_bounds__(256) stream_scalar_kernel(const T *__restrict__ X, const T *__restrict__ V,
                                                             T *__restrict__ Y, long long total, int a, int b,
-                                                            int c, int d) {
+                                                            int c, int d, const T *__restrict__ bias, int act) {
     const long long in_f = (long long)a * c * d, out_f = (long long)a * b * d;
     const long long bd = (long long)b * d;
     const long long stride = (long long)gridDim.x * blockDim.x;
@@ -132,6 +141,7 @@ __global__ void __launch_bounds__(256) stream_scalar_kernel(const T *__restrict_
         const T *v = V + (((long long)i * d + l) * b + k) * c;
         float acc = 0.f;
         for (int j = 0; j < c; ++j) acc = fmaf(to_f(__ldg(v + j)), to_f(__ldg(x + (long long)j * d)), acc);
+        if (bias || act) acc = ep_apply(acc, bias, r, act);  // r = column of this output
         from_f(Y[t], acc);
     }
 }
@@ -155,10 +165,13 @@ __host__ __device__ constexpr int merged_units(int B, int C, int D, int VEC) {
 //          inputs and U*B*d outputs are each one contiguous run; weights
 //          values[i0 .. i0+U)[.][.][.] (contiguous).
 // Threads form a TU x TR grid per CTA: TU consecutive units by TR row lanes.
-template <typename T, int B, int C, int D>
+// EP: fused epilogue (bias and activation) compiled in; the plain
+// instantiation carries none of its code.
+template <typename T, int B, int C, int D, bool EP>
 __global__ void __launch_bounds__(256) stream_reg_kernel(const T *__restrict__ X, const T *__restrict__ V,
                                                          T *__restrict__ Y, long long N, int d, int units,
-                                                         int in_f, int out_f, int tu_log2, int rows_per_cta) {
+                                                         int in_f, int out_f, int tu_log2, int rows_per_cta,
+                                                         const T *__restrict__ bias, int act) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int U = D == 0 ? 1 : merged_units(B, C, D, VEC);
     static_assert(U > 0, "no 16-byte merged layout for this block shape");
@@ -230,6 +243,18 @@ __global__ void __launch_bounds__(256) stream_reg_kernel(const T *__restrict__ X
                 for (int j = 0; j < C; ++j) acc = fmaf(w[(e * B + k) * C + j], xv[e * C + j], acc);
                 yv[e * B + k] = acc;
             }
+        if (EP) {  // fused epilogue; column of (lane e, output k)
+            if (bias) {
+#pragma unroll
+                for (int e = 0; e < NL; ++e)
+#pragma unroll
+                    for (int k = 0; k < B; ++k) {
+                        const int col = D == 0 ? y_off + k * d + e : y_off + (e / D) * (B * D) + k * D + (e % D);
+                        yv[e * B + k] += ep_bias(bias, col);
+                    }
+            }
+            ep_act_array(yv, act);
+        }
         if constexpr (D == 0) {
 #pragma unroll
             for (int k = 0; k < B; ++k) {
@@ -273,9 +298,11 @@ cudaError_t launch_reg(const Problem &p) {
     const long long by = std::max<long long>(1, std::min(max_by, (target + bx - 1) / bx));
     const long long rows_per_cta = (p.batch + by - 1) / by;
     if (bx > INT32_MAX || rows_per_cta > INT32_MAX) return cudaErrorInvalidConfiguration;
-    stream_reg_kernel<T, B, C, D><<<dim3((unsigned)bx, (unsigned)by), 256, 0, p.stream>>>(
+    auto kern = (p.bias || p.act) ? stream_reg_kernel<T, B, C, D, true> : stream_reg_kernel<T, B, C, D, false>;
+    kern<<<dim3((unsigned)bx, (unsigned)by), 256, 0, p.stream>>>(
         static_cast<const T *>(p.X), static_cast<const T *>(p.V), static_cast<T *>(p.Y), p.batch, (int)p.d,
-        (int)units, (int)p.in_features(), (int)p.out_features(), tu_log2, (int)rows_per_cta);
+        (int)units, (int)p.in_features(), (int)p.out_features(), tu_log2, (int)rows_per_cta,
+        static_cast<const T *>(p.bias), p.act);
     return cudaGetLastError();
 }
 
@@ -333,6 +360,7 @@ cudaError_t launch_typed(const Problem &p) {
     const T *X = static_cast<const T *>(p.X);
     const T *V = static_cast<const T *>(p.V);
     T *Y = static_cast<T *>(p.Y);
+    const T *B = static_cast<const T *>(p.bias);
     const cudaError_t er = launch_reg_any<T>(p);
     if (er != cudaErrorNotSupported) return er;
     const bool aligned = (reinterpret_cast<uintptr_t>(p.X) % 16 == 0) && (reinterpret_cast<uintptr_t>(p.Y) % 16 == 0);
@@ -340,14 +368,14 @@ cudaError_t launch_typed(const Problem &p) {
         const long long total = p.batch * p.a * (p.d / VEC);
         if (p.b <= 2)
             stream_vec_kernel<T, 2><<<grid_for(total, 256), 256, 0, p.stream>>>(X, V, Y, total, (int)p.a, (int)p.b,
-                                                                               (int)p.c, (int)p.d);
+                                                                               (int)p.c, (int)p.d, B, p.act);
         else
             stream_vec_kernel<T, 4><<<grid_for(total, 256), 256, 0, p.stream>>>(X, V, Y, total, (int)p.a, (int)p.b,
-                                                                               (int)p.c, (int)p.d);
+                                                                               (int)p.c, (int)p.d, B, p.act);
     } else {
         const long long total = p.batch * p.out_features();
         stream_scalar_kernel<T><<<grid_for(total, 256), 256, 0, p.stream>>>(X, V, Y, total, (int)p.a, (int)p.b,
-                                                                            (int)p.c, (int)p.d);
+                                                                            (int)p.c, (int)p.d, B, p.act);
     }
     return cudaGetLastError();
 }

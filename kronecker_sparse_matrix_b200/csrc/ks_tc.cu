@@ -45,6 +45,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "ks_epilogue.cuh"
 #include "ks_internal.h"
 #include "ks_sm100.cuh"
 
@@ -69,6 +70,8 @@ __host__ __device__ constexpr int chunk_j(int dls) { return dls == 8 ? 16 : 64 /
 __host__ __device__ constexpr int chunk_bytes(int dls) { return kRows * chunk_j(dls) * dls * 2; }
 
 struct TcParams {
+    const __nv_bfloat16 *bias;  // fused epilogue: out_f values or null
+    int act;
     long long N;
     int a, b, c, d;
     int out_f;
@@ -83,7 +86,7 @@ struct TcParams {
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
 };
 
-template <int DLS>
+template <int DLS, bool EP>  // EP: fused bias / activation epilogue compiled in
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap vmap, const TcParams p) {
     constexpr int CTJ = chunk_j(DLS);
@@ -324,6 +327,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                         mbar_arrive(&acc_empty[buf]);
                     }
+                    const int kq = ps * p.bp + oc * kc;  // first k of the chunk
+                    const long long ybase = (long long)i * p.b * p.d + l0;
+                    if (EP && p.bias) {  // fused epilogue on (k = kq + e, l)
+#pragma unroll
+                        for (int l = 0; l < DLS; ++l)
+#pragma unroll
+                            for (int e = 0; e < kChunkElems / DLS; ++e)
+                                if (e < kc) acc[l][e] += ep_bias(p.bias, ybase + (long long)(kq + e) * p.d + l);
+                    }
+                    if (EP && p.act) {
+#pragma unroll
+                        for (int l = 0; l < DLS; ++l) ep_act_array(acc[l], p.act);
+                    }
                     // unit u = elements 8u..8u+7 of (k*DLS + l); box u*8/bi, 16-byte chunk within its row
 #pragma unroll
                     for (int u = 0; u < kChunkElems / 8; ++u) {
@@ -347,8 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     // copy the box out: each warp instruction moves whole 16-byte units of
                     // 32 / units rows (4 rows x 128 contiguous bytes when sw)
-                    const int kq = ps * p.bp + oc * kc;  // first k of the chunk
-                    const long long ybase = (long long)i * p.b * p.d + l0;
                     if (sw) {
                         const int u = lane & 7;
                         const int f = 8 * u;
@@ -530,6 +544,8 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.box_elems = bi;
     p.box_sw128 = sw128 ? 1 : 0;
     p.N = pr.batch;
+    p.bias = static_cast<const __nv_bfloat16 *>(pr.bias);
+    p.act = pr.act;
     p.a = (int)pr.a; p.b = (int)pr.b; p.c = (int)pr.c; p.d = (int)pr.d;
     p.out_f = (int)pr.out_features();
     p.bp = bp;
@@ -551,7 +567,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.off_epi = L.off_epi;
     p.off_bar = L.off_bar;
     p.v_stage_bytes = L.v_stage_bytes;
-    auto kern = tc_kernel<DLS>;
+    auto kern = (pr.bias || pr.act) ? tc_kernel<DLS, true> : tc_kernel<DLS, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (e != cudaSuccess) return e;
     const long long grid = std::min<long long>(p.n_tiles, (long long)sm_count());
