@@ -498,6 +498,15 @@ def extra_configs(args, dev, peaks):
             out[f"{name}-{dt}-{grad}"] = {"pattern": list(p), "batch": n, "us": t * 1e6, "tflops": tf,
                                           "frac": tf / roof}
         del f, dy
+    # hierarchical butterfly factorization of a dense 4096 x 4096 product of
+    # butterfly factors (the producer of the chain's factors)
+    c = inputs.butterfly(device=dev)
+    A = ks.chain(torch.eye(4096, device=dev), c.factors, c.patterns).t().contiguous()
+    t = timed(lambda: ks.butterfly_factorize(A), args.steps)
+    out["butterfly-factorize-4096-fp32"] = {"us": t * 1e6, "gbs": A.numel() * 4 / t / 1e9,
+                                            "note": "rank-one fits of 4096 64x64 blocks at the top split, then "
+                                                    "recursively; bytes = one read of A"}
+    del A, c
     for dt in ("fp32", "bf16"):
         c = inputs.butterfly(device=dev, dtype=torch_dtype(dt))
         s = 4 if dt == "fp32" else 2

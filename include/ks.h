@@ -221,6 +221,24 @@ ks_status ks_chain_noalloc(const void *X, const void *const *factors,
                            const ks_pattern *patterns, int n_factors,
                            int64_t batch, void *Y, int dtype, void *stream);
 
+/* Hierarchical butterfly factorization (the producer of butterfly chains):
+ * fits the 2^log2n x 2^log2n dense matrix A (row-major, the K of Y = X K^T)
+ * with the butterfly factors F_k = (2^(k-1), 2, 2, 2^(log2n-k)), k = 1..log2n,
+ * F_1 applied first, so that ks_chain(X, factors, patterns) ~ X A^T.
+ * The factor range is split in the middle recursively; each split fits two
+ * chainable KS factors to the current KS product block by block with its best
+ * rank-one approximation (power iteration from the block's largest-norm row,
+ * a fixed number of steps).  A product of butterfly factors is recovered
+ * exactly up to rounding; for other matrices the blocks' rank-one fits are
+ * exact only as far as the power iteration has converged.  Each factor's
+ * split sign makes the largest entry of its row part positive.
+ * A and factors[0 .. log2n-1] are DEVICE fp32 arrays (factor k-1 holds
+ * 2^(log2n+1) values [a][d][b][c]); dtype KS_F32 (KS_BF16: KS_ERR_UNSUPPORTED).
+ * 1 <= log2n <= 14.  Intermediates come from the library's pool (stream-
+ * ordered, freed before return). */
+ks_status ks_butterfly_factorize(const void *A, int log2n, void *const *factors,
+                                 int dtype, void *stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char *ks_last_error(void);
 

@@ -127,6 +127,24 @@ def matmul_dv(dy: torch.Tensor, x: torch.Tensor, pattern: Pattern, *, out: Optio
     return out
 
 
+def butterfly_factorize(a: torch.Tensor, *, stream: Optional[torch.cuda.Stream] = None):
+    """Fit a dense 2^L x 2^L fp32 CUDA matrix A (the K of Y = X K^T) with the L
+    butterfly factors; returns (factors, patterns) for chain(), factor 0 first."""
+    if a.dim() != 2 or a.shape[0] != a.shape[1] or not a.is_cuda or not a.is_contiguous():
+        raise ValueError("a must be a square contiguous CUDA matrix")
+    n = a.shape[0]
+    L = n.bit_length() - 1
+    if n != 1 << L or L < 1:
+        raise ValueError("the size must be a power of two")
+    patterns = [(2 ** (k - 1), 2, 2, 2 ** (L - k)) for k in range(1, L + 1)]
+    factors = [torch.empty(p[0] * p[1] * p[2] * p[3], dtype=a.dtype, device=a.device) for p in patterns]
+    ptrs = (ctypes.c_void_p * L)(*[f.data_ptr() for f in factors])
+    with torch.cuda.device(a.device):
+        st = _lib.load().ks_butterfly_factorize(a.data_ptr(), L, ptrs, ks_dtype_of(a), _stream_ptr(stream, a.device))
+    _lib.check(st)
+    return factors, patterns
+
+
 class _KSLinearFn(torch.autograd.Function):
     """Y = X K^T with K the KS factor of `pattern`; both gradients on the GPU."""
 

@@ -42,6 +42,7 @@ SIGNATURES = {
     "ks_matmul_ep": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp, _int, _int, _vp]),
     "ks_chain_ep": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp,
                            _int, _vp]),
+    "ks_butterfly_factorize": (_int, [_vp, _int, ctypes.POINTER(_vp), _int, _vp]),
     "ks_matmul_dx": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_matmul_dv": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_chain_ex": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp]),

@@ -444,6 +444,76 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int6
     return result == KS_OK ? ok() : result;
 }
 
+namespace {
+
+// The product of butterfly factors F_p .. F_q of size 2^L (F_k = (2^(k-1), 2, 2, 2^(L-k))).
+ks_pattern butterfly_range(int p, int q, int L) {
+    return ks_pattern{1LL << (p - 1), 1LL << (q - p + 1), 1LL << (q - p + 1), 1LL << (L - q)};
+}
+
+// Splits the range [p, q], whose product values are P, in the middle and fits
+// the two halves; recurses until single factors land in factors[k - 1].
+ks_status factorize_range(const float *P, int p, int q, int L, float *const *factors, cudaMemPool_t pool,
+                          cudaStream_t st) {
+    const int r = (p + q - 1) / 2;
+    const ks_pattern p1 = butterfly_range(p, r, L), p2 = butterfly_range(r + 1, q, L);
+    const int64_t n1 = p1.a * p1.b * p1.c * p1.d, n2 = p2.a * p2.b * p2.c * p2.d;
+    float *v1 = nullptr, *v2 = nullptr;
+    ks_status result = KS_OK;
+    if (r == p) {
+        v1 = factors[p - 1];
+    } else if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&v1), (size_t)n1 * 4, pool, st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "factorization workspace of %lld bytes", (long long)(n1 * 4));
+    }
+    if (r + 1 == q) {
+        v2 = factors[q - 1];
+    } else if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&v2), (size_t)n2 * 4, pool, st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        result = fail(KS_ERR_ALLOC, "factorization workspace of %lld bytes", (long long)(n2 * 4));
+    }
+    if (result == KS_OK) {
+        const cudaError_t e = launch_rank1_fit(P, v1, v2, p1.a, p1.b, p1.c, p2.b, p2.c, p2.d, st);
+        if (e != cudaSuccess) result = cuda_fail(e, "rank-one fit launch");
+    }
+    if (result == KS_OK && r > p) result = factorize_range(v1, p, r, L, factors, pool, st);
+    if (result == KS_OK && q > r + 1) result = factorize_range(v2, r + 1, q, L, factors, pool, st);
+    if (r != p && v1) (void)cudaFreeAsync(v1, st);
+    if (r + 1 != q && v2) (void)cudaFreeAsync(v2, st);
+    return result;
+}
+
+}  // namespace
+
+ks_status ks_butterfly_factorize(const void *A, int log2n, void *const *factors, int dtype, void *stream) {
+    if (dtype != KS_F32 && dtype != KS_TF32)
+        return fail(dtype == KS_BF16 ? KS_ERR_UNSUPPORTED : KS_ERR_INVALID_ARG,
+                    "the factorization runs on fp32 matrices only (dtype %d)", dtype);
+    if (log2n < 1 || log2n > 14) return fail(KS_ERR_INVALID_ARG, "log2n must be in 1..14 (got %d)", log2n);
+    if (!A || !factors) return fail(KS_ERR_INVALID_ARG, "A and factors must be non-null");
+    ks_status s;
+    if ((s = check_align(A, 4, "A")) != KS_OK) return s;
+    const int64_t N = 1LL << log2n;
+    for (int k = 0; k < log2n; ++k) {
+        if (!factors[k]) return fail(KS_ERR_INVALID_ARG, "factor %d is null", k);
+        if ((s = check_align(factors[k], 4, "a factor")) != KS_OK) return s;
+        if (ranges_overlap(factors[k], 2 * N * 4, A, N * N * 4)) return fail(KS_ERR_INVALID_ARG, "factor %d overlaps A", k);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (log2n == 1) {  // a single factor (1, 2, 2, 1) holds A itself
+        const cudaError_t e = cudaMemcpyAsync(factors[0], A, 4 * 4, cudaMemcpyDeviceToDevice, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "copy");
+    }
+    cudaMemPool_t pool = chain_pool();
+    if (!pool) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
+    }
+    float *const *f = reinterpret_cast<float *const *>(factors);
+    const ks_status r = factorize_range(static_cast<const float *>(A), 1, log2n, log2n, f, pool, st);
+    return r == KS_OK ? ok() : r;
+}
+
 const char *ks_last_error(void) { return g_msg; }
 
 const char *ks_status_string(int status) {

@@ -82,6 +82,14 @@ cudaError_t launch_dv(const DvProblem &q, float *W, int splits, long long rows_p
 // vt[blk][j][k] = v[blk][k][j] for `blocks` blocks of b x c (KS values transposed per (i, l)).
 cudaError_t launch_transpose_blocks(const void *v, void *vt, int64_t blocks, int64_t b, int64_t c, int dtype,
                                     cudaStream_t stream);
+// Two-factor fit of a KS product (ks_factorize.cu): P of pattern
+// (a1, b1*b2, c1*c2, d2) -> V1 (a1, b1, c1, c2*d2) and V2 (a1*b1, b2, c2, d2),
+// one best rank-one block per (i1, k1, j2, l2).  cudaErrorInvalidValue when a
+// block (b2 x (c1 + 1) floats) exceeds fit_max_block_elems().
+int fit_max_block_elems();
+cudaError_t launch_rank1_fit(const float *P, float *V1, float *V2, int64_t a1, int64_t b1, int64_t c1, int64_t b2,
+                             int64_t c2, int64_t d2, cudaStream_t stream);
+
 // The library's retaining workspace pool of the current device (ks_api.cu).
 cudaMemPool_t chain_pool();
 
