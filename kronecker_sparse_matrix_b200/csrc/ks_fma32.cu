@@ -9,8 +9,8 @@
 // k x DL consecutive l for one block i, accumulated in registers over all j;
 // each warp owns one l and a 64 x (4*TN) piece, each thread 8 rows x TN
 // values of k.  Operands reach shared memory without passing through
-// registers, in a 3-stage ring of 8 j per stage whose copies run ahead of the
-// compute, across tile boundaries too:
+// registers, in a ring of 3 stages (4 for DL = 4) of 8 j per stage whose
+// copies run ahead of the compute, across tile boundaries too:
 //
 //   X       16-byte cp.async of whole row segments, kept in X's own order:
 //           As[n][j*DL + l] (row stride RA = 8*DL + 4 words, RA/4 odd);
@@ -36,7 +36,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kJT = 8;   // j per stage
-constexpr int kNS = 3;   // ring stages
 
 struct Fma32Params {
     const float *X;
@@ -65,9 +64,13 @@ struct Tile32 {
     static constexpr int RS = DL * BKP + (DL == 1 ? 0 : 4);  // epilogue row stride, = 4 (mod 8)
     // the epilogue stages all rows at once if that fits beside the ring, else
     // half of each warp's 64 rows per pass
-    static constexpr int NP = (kNS * STAGE + BM * RS) * 4 <= 232448 ? 1 : 2;
+    // ring depth: 3 stages; 4 for DL = 4, the one l width a fourth stage made
+    // faster (elsewhere it was slower: the larger shared-memory carve-out
+    // leaves less L1 for the 4-byte values copies)
+    static constexpr int NS = (DL == 4 && (4 * STAGE + BM / 2 * RS) * 4 <= 232448) ? 4 : 3;
+    static constexpr int NP = (NS * STAGE + BM * RS) * 4 <= 232448 ? 1 : 2;
     static constexpr int EPI = BM / NP * RS;
-    static constexpr int SMEM_FLOATS = kNS * STAGE + EPI;
+    static constexpr int SMEM_FLOATS = NS * STAGE + EPI;
     static constexpr int CA = 2 * DL;                 // 16-byte chunks per A row per stage
     static constexpr int NXC = (BM * CA + kThreads - 1) / kThreads;      // A copies per thread
     static constexpr int NV = (DL * BKL * kJT + kThreads - 1) / kThreads;  // values copies per thread
@@ -96,6 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
     using TL = Tile32<DL, WM, WK, TN>;
     constexpr int BM = TL::BM, BKL = TL::BKL;
     extern __shared__ __align__(16) float smem[];
+    constexpr int kNS = TL::NS;
     float *sEpi = smem + kNS * TL::STAGE;
     const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(smem);
 
