@@ -164,6 +164,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t sbo)
            (1ull << 46) | (2ull << 61);
 }
 
+// Shared-memory matrix descriptor for a swizzled K-major operand: `layout` is
+// the tcgen05 layout type (2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle),
+// SBO the stride between 8-row groups; LBO is unused (16 bytes).  The atoms
+// (8 rows x the swizzle width) must sit at addresses aligned to their size; a
+// K step inside an atom advances `addr` by 32 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw(uint32_t addr, uint32_t sbo, uint32_t layout) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46) | ((uint64_t)layout << 61);
+}
+
 // AND of `ok` over the `count` threads of named barrier `id` (all of them
 // must call it).  Used to keep the loader warps' decisions uniform.
 __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool ok) {

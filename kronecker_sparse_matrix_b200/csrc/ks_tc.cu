@@ -68,6 +68,12 @@ constexpr int kSmemLimit = 232448; // per-block opt-in maximum on sm_100
 // j per X chunk and chunk bytes, per DLS
 __host__ __device__ constexpr int chunk_j(int dls) { return dls == 8 ? 16 : 64 / dls; }
 __host__ __device__ constexpr int chunk_bytes(int dls) { return kRows * chunk_j(dls) * dls * 2; }
+// The values of one chunk land as DLS planes of bp rows (k) x chunk_j(dls) j,
+// K-major with the swizzle as wide as a row (2 * chunk_j bytes): tcgen05
+// layout type and the TMA swizzle mode for that width.
+__host__ __device__ constexpr uint32_t v_layout(int dls) {
+    return chunk_j(dls) == 64 ? 2u : chunk_j(dls) == 32 ? 4u : 6u;
+}
 
 struct TcParams {
     const __nv_bfloat16 *bias;  // fused epilogue: out_f values or null
@@ -84,6 +90,7 @@ struct TcParams {
     int off_v, off_epi, off_bar;     // shared-memory carve-up (ring at offset 0)
     int v_stage_bytes;
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
+    int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
 template <int DLS, bool EP>  // EP: fused bias / activation epilogue compiled in
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = mbar_wait(&x_empty[xs], ((xq / S) & 1) ^ 1, abort_flag, p.status);
                         if (!ok) break;
                         mbar_expect_tx(&x_full[xs], (uint32_t)CB);
-                        if (DLS == 8)
+                        if (DLS == 8 && !p.x3d)
                             tma_load_4d(sR + xs * CB, &xmap, &x_full[xs], l0, ch * CTJ, i, n0);
                         else
                             tma_load_3d(sR + xs * CB, &xmap, &x_full[xs], ch * CTJ * p.d, i, n0);
@@ -163,8 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = mbar_wait(&v_empty[vs], ((vq / VS) & 1) ^ 1, abort_flag, p.status);
                         if (!ok) break;
                         mbar_expect_tx(&v_full[vs], (uint32_t)p.v_stage_bytes);
-                        tma_load_4d(sV + vs * p.v_stage_bytes, &vmap, &v_full[vs], 0, ps * p.bp, ch * (CTJ / 8),
-                                    i * p.d + l0);
+                        tma_load_3d(sV + vs * p.v_stage_bytes, &vmap, &v_full[vs], ch * CTJ, ps * p.bp, i * p.d + l0);
                         ++vq;
                     }
                 }
@@ -216,9 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     ad = smem_desc_sw128(stage + sl * 32, 1024);
                                 else
                                     ad = smem_desc(stage + l * (CTJ * 256) + sl * 2 * 2048, 2048, 128);
-                                // values stage: [l][CTJ/8 j-groups][bp k][8 j], K step = two j-groups
-                                const uint32_t b_addr = vstage + l * (p.bp * CTJ * 2) + sl * 2 * (p.bp * 16);
-                                const uint64_t bd = smem_desc(b_addr, p.bp * 16, 128);
+                                // values stage: [l][bp k][CTJ j] swizzled rows, K step = 32 bytes
+                                const uint32_t b_addr = vstage + l * (p.bp * CTJ * 2) + sl * 32;
+                                const uint64_t bd = smem_desc_sw(b_addr, 8 * CTJ * 2, v_layout(DLS));
                                 mma_bf16(d_base + l * p.bp, ad, bd, idesc, s > 0 ? 1u : 0u);
                             }
                         }
@@ -504,7 +510,8 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap xmap, vmap;
     CUresult r;
-    if (DLS == 8) {
+    const bool x3d = DLS < 8 || pr.d == 8;
+    if (!x3d) {
         // X as (d, c, a, N): a box (8 l, 16 j, 1, 128 rows) = [row][j][l]
         cuuint64_t dims[4] = {(cuuint64_t)pr.d, (cuuint64_t)pr.c, (cuuint64_t)pr.a, (cuuint64_t)pr.batch};
         cuuint64_t strides[3] = {(cuuint64_t)pr.d * 2, (cuuint64_t)pr.c * pr.d * 2, (cuuint64_t)pr.in_features() * 2};
@@ -513,24 +520,31 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        // X as (c*d, a, N): a box (64 elements, 1, 128 rows) = [row][(j, l)];
-        // for d == 1 with the 128-byte swizzle, the K-major operand tile itself
+        // X as (c*d, a, N): a box (CTJ*DLS elements, 1, 128 rows) = [row][(j, l)]
+        // (d == DLS, or d == 8: whole 256-byte rows); for d == 1 with the
+        // 128-byte swizzle, the K-major operand tile itself
         cuuint64_t dims[3] = {(cuuint64_t)(pr.c * pr.d), (cuuint64_t)pr.a, (cuuint64_t)pr.batch};
         cuuint64_t strides[2] = {(cuuint64_t)pr.c * pr.d * 2, (cuuint64_t)pr.in_features() * 2};
-        cuuint32_t box[3] = {64, 1, (cuuint32_t)kRows};
+        cuuint32_t box[3] = {(cuuint32_t)(chunk_j(DLS) * DLS), 1, (cuuint32_t)kRows};
         r = encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pr.X), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, DLS == 1 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     }
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     {
-        // values[i][l][k][j] viewed as (j%8, k, j/8, i*d+l): a box (8, bp, CTJ/8, DLS)
-        // lands as [l][j/8][k][8 j], K-major core matrices for CTJ/16 K steps.
-        cuuint64_t dims[4] = {8, (cuuint64_t)pr.b, (cuuint64_t)(pr.c / 8), (cuuint64_t)(pr.a * pr.d)};
-        cuuint64_t strides[3] = {(cuuint64_t)pr.c * 2, 16, (cuuint64_t)pr.b * pr.c * 2};
-        cuuint32_t box[4] = {8, (cuuint32_t)bp, (cuuint32_t)(chunk_j(DLS) / 8), (cuuint32_t)DLS};
-        r = encode(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pr.V), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        // values[i][l][k][j] viewed as (j, k, i*d+l): a box (CTJ j, bp k, DLS l)
+        // lands as DLS planes [k][CTJ j], rows of 2*CTJ bytes swizzled at that
+        // width: the K-major operand for CTJ/16 K steps.  (A TMA fetches about
+        // one box row per clock, so rows of 16 bytes would cap the copy far
+        // below the bandwidth this kernel needs.)
+        cuuint64_t dims[3] = {(cuuint64_t)pr.c, (cuuint64_t)pr.b, (cuuint64_t)(pr.a * pr.d)};
+        cuuint64_t strides[2] = {(cuuint64_t)pr.c * 2, (cuuint64_t)pr.b * pr.c * 2};
+        cuuint32_t box[3] = {(cuuint32_t)chunk_j(DLS), (cuuint32_t)bp, (cuuint32_t)DLS};
+        const CUtensorMapSwizzle vsw = chunk_j(DLS) == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : chunk_j(DLS) == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                            : CU_TENSOR_MAP_SWIZZLE_32B;
+        r = encode(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pr.V), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, vsw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
@@ -543,6 +557,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     TcParams p;
     p.box_elems = bi;
     p.box_sw128 = sw128 ? 1 : 0;
+    p.x3d = x3d ? 1 : 0;
     p.N = pr.batch;
     p.bias = static_cast<const __nv_bfloat16 *>(pr.bias);
     p.act = pr.act;
