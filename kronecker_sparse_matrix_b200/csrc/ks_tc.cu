@@ -68,6 +68,16 @@ constexpr int kSmemLimit = 232448; // per-block opt-in maximum on sm_100
 // j per X chunk and chunk bytes, per DLS
 __host__ __device__ constexpr int chunk_j(int dls) { return dls == 8 ? 16 : 64 / dls; }
 __host__ __device__ constexpr int chunk_bytes(int dls) { return kRows * chunk_j(dls) * dls * 2; }
+// Transposed operand planes (DLS > 1): MN-major core matrices of 8 j x 8 rows
+// (128 bytes), the 16 row groups of a j octet 144 bytes apart (one 16-byte
+// pad each), so that the transposer's 16-byte stores from one warp spread
+// over all eight bank groups; j octets are 16 * 144 bytes apart.
+constexpr int kGroupStride = 144;
+constexpr int kOctetStride = 16 * kGroupStride;
+// ring slot: the raw chunk, transposed in place into padded planes
+__host__ __device__ constexpr int slot_bytes(int dls) {
+    return dls == 1 ? chunk_bytes(1) : dls * (chunk_j(dls) / 8) * kOctetStride;
+}
 // The values of one chunk land as DLS planes of bp rows (k) x chunk_j(dls) j,
 // K-major with the swizzle as wide as a row (2 * chunk_j bytes): tcgen05
 // layout type and the TMA swizzle mode for that width.
@@ -90,6 +100,7 @@ struct TcParams {
     int off_v, off_epi, off_bar;     // shared-memory carve-up (ring at offset 0)
     int v_stage_bytes;
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
+    int box_row_bytes;               // staging row stride when not swizzled (an odd number of 16-byte units)
     int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
@@ -98,11 +109,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap vmap, const TcParams p) {
     constexpr int CTJ = chunk_j(DLS);
     constexpr int CB = chunk_bytes(DLS);
+    constexpr int SB = slot_bytes(DLS);
     constexpr int UNITS = CTJ * DLS / 8;    // 16-byte units per row of a chunk (8 or 16)
     constexpr int TASKS = 16 * UNITS / 128; // transpose tasks per loader thread (1 or 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sR = smem;  // X ring: stage s at s * CB (1024-aligned)
+    uint8_t *sR = smem;  // X ring: stage s at s * SB (1024-aligned)
     uint8_t *sV = smem + p.off_v;
     uint8_t *sE = smem + p.off_epi;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.off_bar);
@@ -161,9 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         mbar_expect_tx(&x_full[xs], (uint32_t)CB);
                         if (DLS == 8 && !p.x3d)
-                            tma_load_4d(sR + xs * CB, &xmap, &x_full[xs], l0, ch * CTJ, i, n0);
+                            tma_load_4d(sR + xs * SB, &xmap, &x_full[xs], l0, ch * CTJ, i, n0);
                         else
-                            tma_load_3d(sR + xs * CB, &xmap, &x_full[xs], ch * CTJ * p.d, i, n0);
+                            tma_load_3d(sR + xs * SB, &xmap, &x_full[xs], ch * CTJ * p.d, i, n0);
                         ++xq;  // counted as soon as it is in flight (the abort drain relies on it)
                         // the values of the same CTJ j: values[i, l0:l0+DLS, pass k's, chunk j's]
                         const int vs = vq % VS;
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++vq;
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t stage = su32(sR) + xs * CB;
+                        const uint32_t stage = su32(sR) + xs * SB;
                         const uint32_t vstage = su32(sV) + vs * p.v_stage_bytes;
                         for (int s = ch * CTJ / kStepJ; s < n_steps && s < (ch + 1) * CTJ / kStepJ; ++s) {
                             const int sl = s - ch * CTJ / kStepJ;  // K step within the chunk
@@ -221,7 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (DLS == 1)
                                     ad = smem_desc_sw128(stage + sl * 32, 1024);
                                 else
-                                    ad = smem_desc(stage + l * (CTJ * 256) + sl * 2 * 2048, 2048, 128);
+                                    ad = smem_desc(stage + l * (CTJ / 8) * kOctetStride + sl * 2 * kOctetStride,
+                                                   kOctetStride, kGroupStride);
                                 // values stage: [l][bp k][CTJ j] swizzled rows, K step = 32 bytes
                                 const uint32_t b_addr = vstage + l * (p.bp * CTJ * 2) + sl * 32;
                                 const uint64_t bd = smem_desc_sw(b_addr, 8 * CTJ * 2, v_layout(DLS));
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool w = mbar_wait(&x_full[xs], (xq / S) & 1, abort_flag, p.status);
                         ok = bar_and(1, 128, w);  // uniform over the four loader warps
                         if (!ok) break;
-                        uint8_t *st = sR + xs * CB;
+                        uint8_t *st = sR + xs * SB;
                         uint4 out[TASKS][8];
 #pragma unroll
                         for (int k = 0; k < TASKS; ++k) {
@@ -272,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int e = 0; e < 8; ++e) {
                                 const int f = 8 * q + e;
                                 const int j = f / DLS, l = f % DLS;  // j within the chunk
-                                *reinterpret_cast<uint4 *>(st + l * (CTJ * 256) + (j >> 3) * 2048 + g8 * 128 +
-                                                           (j & 7) * 16) = out[k][e];
+                                *reinterpret_cast<uint4 *>(st + (l * (CTJ / 8) + (j >> 3)) * kOctetStride +
+                                                           g8 * kGroupStride + (j & 7) * 16) = out[k][e];
                             }
                         }
                         fence_proxy_async();
@@ -296,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kc = p.kc;                      // k per chunk
         const int n_oc = p.bp / kc;
         const int units = DLS * kc / 8;           // 16-byte output units per row per chunk
-        const int bi = p.box_elems;               // elements per TMA store box row
         const bool sw = p.box_sw128 != 0;
+        const int rsb = p.box_row_bytes;          // staging row stride (not sw)
         uint32_t accq = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
@@ -356,41 +369,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const int f0 = 8 * u + 2 * h, f1 = f0 + 1;
                                 w[h] = pack_bf16x2(acc[f0 % DLS][f0 / DLS], acc[f1 % DLS][f1 / DLS]);
                             }
-                            uint32_t off;
-                            if (sw) {
-                                const int bx = u >> 3, c16 = u & 7;
-                                off = bx * 4096 + lane * 128 + ((c16 ^ (lane & 7)) << 4);
-                            } else {
-                                off = lane * (bi * 2) + u * 16;
-                            }
+                            const uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
                             *reinterpret_cast<uint4 *>(stage + off) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
                     __syncwarp();
-                    // copy the box out: each warp instruction moves whole 16-byte units of
-                    // 32 / units rows (4 rows x 128 contiguous bytes when sw)
-                    if (sw) {
+                    // copy the box out: lane = (row r = lane / 8 + 4 t, unit u = lane % 8), so each
+                    // warp instruction moves whole 16-byte units of four rows (four full 128-byte row
+                    // segments when sw); lanes past the row's units idle
+                    {
                         const int u = lane & 7;
-                        const int f = 8 * u;
-                        const long long col = ybase + (long long)(kq + f / DLS) * p.d + f % DLS;
+                        if (u < units) {
+                            const int f = 8 * u;
+                            const long long col = ybase + (long long)(kq + f / DLS) * p.d + f % DLS;
+                            int r = lane >> 3;
+                            __nv_bfloat16 *yp = p.Y + (long long)(row0 + r) * p.out_f + col;
+                            const long long ystep = 4LL * p.out_f;
+                            const int rows_here = (int)min(p.N - (long long)row0, 32LL);
 #pragma unroll
-                        for (int r = lane >> 3; r < 32; r += 4) {
-                            const int row = row0 + r;
-                            if (row < p.N) {
-                                const uint4 val =
-                                    *reinterpret_cast<const uint4 *>(stage + r * 128 + ((u ^ (r & 7)) << 4));
-                                *reinterpret_cast<uint4 *>(p.Y + (long long)row * p.out_f + col) = val;
-                            }
-                        }
-                    } else {
-                        for (int idx = lane; idx < 32 * units; idx += 32) {
-                            const int r = idx / units, u = idx - r * units;
-                            const int row = row0 + r;
-                            if (row < p.N) {
-                                const int f = 8 * u;
-                                const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * (bi * 2) + u * 16);
-                                *reinterpret_cast<uint4 *>(p.Y + (long long)row * p.out_f + ybase +
-                                                           (long long)(kq + f / DLS) * p.d + f % DLS) = val;
+                            for (int t = 0; t < 8; ++t, r += 4, yp += ystep) {
+                                if (r < rows_here) {
+                                    const uint32_t soff = sw ? r * 128 + ((u ^ (r & 7)) << 4) : r * rsb + u * 16;
+                                    *reinterpret_cast<uint4 *>(yp) = *reinterpret_cast<const uint4 *>(stage + soff);
+                                }
                             }
                         }
                     }
@@ -458,7 +459,7 @@ constexpr int kBarBytes = (3 * kMaxStages + 2 * kVStages + 2 + 2 + 1) * 8 + 16;
 bool tc_layout(int dls, int bp, TcLayout *out) {
     TcLayout L;
     auto up = [](int x, int a) { return (x + a - 1) / a * a; };
-    const int cb = chunk_bytes(dls);
+    const int cb = slot_bytes(dls);
     L.v_stage_bytes = 2 * bp * chunk_j(dls) * dls;
     const int epi = 4 * kEpiWarpBytes;
     const int budget = kSmemLimit - 2048 - epi - kBarBytes;  // alignment slack
@@ -557,6 +558,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     TcParams p;
     p.box_elems = bi;
     p.box_sw128 = sw128 ? 1 : 0;
+    p.box_row_bytes = bi * 2 + ((bi / 8) % 2 == 0 ? 16 : 0);
     p.x3d = x3d ? 1 : 0;
     p.N = pr.batch;
     p.bias = static_cast<const __nv_bfloat16 *>(pr.bias);
