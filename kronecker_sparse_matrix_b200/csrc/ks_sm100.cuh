@@ -174,6 +174,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw(uint32_t addr, uint32_t sbo, ui
            (1ull << 46) | ((uint64_t)layout << 61);
 }
 
+// TMA tensor store of a 2-D box from shared memory (bulk group of this
+// thread); x is the element column (x * element size a multiple of 16 bytes),
+// y the row.  Rows past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t ssrc, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(ssrc)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk copies have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's bulk copies are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // AND of `ok` over the `count` threads of named barrier `id` (all of them
 // must call it).  Used to keep the loader warps' decisions uniform.
 __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool ok) {

@@ -43,6 +43,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "ks_epilogue.cuh"
@@ -101,12 +102,14 @@ struct TcParams {
     int v_stage_bytes;
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
     int box_row_bytes;               // staging row stride when not swizzled (an odd number of 16-byte units)
+    int ytma;                        // the swizzled staging box goes to Y as one TMA store (d == DLS)
     int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
 template <int DLS, bool EP>  // EP: fused bias / activation epilogue compiled in
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap vmap, const TcParams p) {
+    tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap vmap,
+              const __grid_constant__ CUtensorMap ymap, const TcParams p) {
     constexpr int CTJ = chunk_j(DLS);
     constexpr int CB = chunk_bytes(DLS);
     constexpr int SB = slot_bytes(DLS);
@@ -310,7 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_oc = p.bp / kc;
         const int units = DLS * kc / 8;           // 16-byte output units per row per chunk
         const bool sw = p.box_sw128 != 0;
-        const int rsb = p.box_row_bytes;          // staging row stride (not sw)
+        // staging row stride (not sw): dense rows for the tensor store, else padded rows
+        const int rsb = p.ytma ? p.box_elems * 2 : p.box_row_bytes;
         uint32_t accq = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
@@ -359,6 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int l = 0; l < DLS; ++l) ep_act_array(acc[l], p.act);
                     }
+                    if (p.ytma) {  // the previous box store has finished reading the staging
+                        if (lane == 0) bulk_wait_read_all();
+                        __syncwarp();
+                    }
                     // unit u = elements 8u..8u+7 of (k*DLS + l); box u*8/bi, 16-byte chunk within its row
 #pragma unroll
                     for (int u = 0; u < kChunkElems / 8; ++u) {
@@ -372,6 +380,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
                             *reinterpret_cast<uint4 *>(stage + off) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
+                    }
+                    if (p.ytma) {
+                        // d == DLS: the box is 32 rows x DLS*kc contiguous elements of Y at column
+                        // ybase + kq*d (staged in the TMA's 128-byte swizzle when rows are 128 bytes,
+                        // densely otherwise); one thread hands it to the tensor store (rows past N
+                        // are clipped by the tensor map)
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0 && (long long)row0 < p.N) {
+                            tma_store_2d(&ymap, su32(stage), (int)(ybase + (long long)kq * p.d), row0);
+                            bulk_commit();
+                        }
+                        continue;
                     }
                     __syncwarp();
                     // copy the box out: lane = (row r = lane / 8 + 4 t, unit u = lane % 8), so each
@@ -401,6 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    // the box stores issued by this warp's lane 0 are complete before the CTA
+    // (and its shared memory) goes away
+    if (warp >= kEpiWarp0 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -550,6 +574,22 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
     // epilogue chunk: kc k's; rows of 64 elements use the swizzled staging box
+    const int kc0 = tc_kc(DLS, bp);
+    const bool ytma = pr.d == DLS && (reinterpret_cast<uintptr_t>(pr.Y) % 16) == 0;
+    CUtensorMap ymap;
+    memset(&ymap, 0, sizeof(ymap));
+    if (ytma) {
+        // Y as (out_f, N): a box (DLS*kc elements, 32 rows); 64-element rows with the
+        // 128-byte swizzle of the staging, shorter rows packed densely
+        const bool sw = DLS * kc0 == kChunkElems;
+        cuuint64_t dims[2] = {(cuuint64_t)pr.out_features(), (cuuint64_t)pr.batch};
+        cuuint64_t strides[1] = {(cuuint64_t)pr.out_features() * 2};
+        cuuint32_t box[2] = {(cuuint32_t)(DLS * kc0), 32};
+        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.Y, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     const int kc = tc_kc(DLS, bp);
     if (kc == 0) return cudaErrorInvalidConfiguration;
     const bool sw128 = (DLS * kc) == kChunkElems;
@@ -559,6 +599,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.box_elems = bi;
     p.box_sw128 = sw128 ? 1 : 0;
     p.box_row_bytes = bi * 2 + ((bi / 8) % 2 == 0 ? 16 : 0);
+    p.ytma = ytma ? 1 : 0;
     p.x3d = x3d ? 1 : 0;
     p.N = pr.batch;
     p.bias = static_cast<const __nv_bfloat16 *>(pr.bias);
@@ -588,7 +629,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (e != cudaSuccess) return e;
     const long long grid = std::min<long long>(p.n_tiles, (long long)sm_count());
-    kern<<<(int)grid, kThreads, L.total, pr.stream>>>(xmap, vmap, p);
+    kern<<<(int)grid, kThreads, L.total, pr.stream>>>(xmap, vmap, ymap, p);
     return cudaGetLastError();
 }
 
