@@ -5,21 +5,26 @@
 // (taxoreview.com page on Kronecker-sparse matrix multiplication, first
 // abstract: a fused, output-stationary kernel with no permutation passes).
 //
-// The tile is the one of ks_fma.cu: BM = 64*WM rows x BKL = 4*TN*WK values of
-// k x DL consecutive l for one block i, accumulated in registers over all j;
-// each warp owns one l and a 64 x (4*TN) piece, each thread 8 rows x TN
-// values of k.  Operands reach shared memory without passing through
-// registers, in a ring of 3 stages (4 for DL = 4) of 8 j per stage whose
-// copies run ahead of the compute, across tile boundaries too:
+// A tile is BM rows x BKL values of k x DL consecutive l of one block i,
+// accumulated in registers over all j.  Every warp spans all DL l of its
+// tile: its 32 lanes are RG row groups x DL values of l x KQ groups of k
+// (KQ = 1, 1, 2, 4 and RG = 4, 8, 8, 8 for DL = 8, 4, 2, 1), and a thread owns
+// 8 rows (rg + RG*m) x TN values of k (4 consecutive per group) of one l.  The
+// outputs Y[n][k*d + l0 .. l0+DL-1] of a row and k thus sit in neighbouring
+// lanes and leave straight from registers: no shared-memory interleave of
+// the l, no barrier after a tile.  Operands reach shared memory without passing
+// through registers, in a ring of stages of 8 j whose copies run ahead of the
+// compute, across tile boundaries too:
 //
 //   X       16-byte cp.async of whole row segments, kept in X's own order:
-//           As[n][j*DL + l] (row stride RA = 8*DL + 4 words, RA/4 odd);
+//           As[n][j*DL + l], row stride RA chosen so that one warp's loads
+//           (RG rows x DL l) fall in distinct banks;
 //   values  4-byte cp.async into Bs[l][j][k] (k contiguous), lanes = 8 j x 4 k
-//           so every copy warp-instruction hits 32 distinct banks.
+//           so every copy warp-instruction hits 32 distinct banks; or, from a
+//           per-call transposed copy, 16-byte copies.  The l planes are PSB
+//           words apart so that one warp's DL (x KQ) 16-byte loads are distinct.
 //
-// A thread's rows are interleaved (lane_r + 8 m), so its 8 scalar loads of A
-// per j hit 8 distinct banks; its k are 4 consecutive per 16, read as float4.
-// Products use fma.rn.f32x2, on pairs of k (DL == 1) or pairs of rows.
+// Products use fma.rn.f32x2 on pairs of k, the X value broadcast.
 //
 // Rounding: every product and sum is an fp32 fma.rn, j = 0..c-1 per output.
 #include <cuda_runtime.h>
@@ -51,30 +56,50 @@ struct Fma32Params {
     int n_tiles;
 };
 
+// Lane geometry per l width: KQ lane groups along k, RG along rows; RA is the
+// As row stride (words): RA*rg + l over a warp's RG x DL loads hits 32
+// distinct banks (or 16 distinct pairs for DL = 2), and rows stay 16-byte
+// aligned for the copies.
+template <int DL>
+struct Lanes32 {
+    static constexpr int KQ = DL == 2 ? 2 : DL == 1 ? 4 : 1;
+    static constexpr int RG = 32 / (DL * KQ);
+    static constexpr int RA = DL == 8 ? 72 : DL == 4 ? 36 : DL == 2 ? 20 : 12;
+};
+
 template <int DL, int WM, int WK, int TN>
 struct Tile32 {
-    static_assert(DL * WM * WK == 8, "8 warps per CTA");
-    static constexpr int BM = 64 * WM;
-    static constexpr int BKL = 4 * TN * WK;
-    static constexpr int RA = kJT * DL + 4;           // As row stride (words), RA/4 odd
+    using LN = Lanes32<DL>;
+    static_assert(WM * WK == 8, "8 warps per CTA");
+    static_assert(TN % 4 == 0, "k per thread in groups of 4");
+    static constexpr int BM = 8 * LN::RG * WM;        // rows per tile (a warp: 8 row groups)
+    static constexpr int KW = LN::KQ * TN;            // k per warp
+    static constexpr int BKL = KW * WK;               // k per tile
+    static constexpr int RA = LN::RA;
     static constexpr int A_WORDS = BM * RA;
     static constexpr int BKP = BKL + 4;               // Bs j-row stride, = 4 (mod 32) or 20
-    static constexpr int PSB = kJT * BKP + 4;         // Bs plane stride
+    // plane stride: PSB/4 odd (DL = 8, 4) or = 2 (mod 8) (DL = 2, with the k pair of lanes)
+    static constexpr int PSB = kJT * BKP + (DL == 2 ? 8 : 4);
     static constexpr int STAGE = A_WORDS + DL * PSB;  // words
-    static constexpr int RS = DL * BKP + (DL == 1 ? 0 : 4);  // epilogue row stride, = 4 (mod 8)
-    // the epilogue stages all rows at once if that fits beside the ring, else
-    // half of each warp's 64 rows per pass
-    // ring depth: 3 stages; 4 for DL = 4, the one l width a fourth stage made
-    // faster (elsewhere it was slower: the larger shared-memory carve-out
-    // leaves less L1 for the 4-byte values copies)
-    static constexpr int NS = (DL == 4 && (4 * STAGE + BM / 2 * RS) * 4 <= 232448) ? 4 : 3;
-    static constexpr int NP = (NS * STAGE + BM * RS) * 4 <= 232448 ? 1 : 2;
-    static constexpr int EPI = BM / NP * RS;
-    static constexpr int SMEM_FLOATS = NS * STAGE + EPI;
+    static constexpr int NS = (4 * STAGE * 4 <= 232448) ? 4 : 3;
+    static constexpr int SMEM_FLOATS = NS * STAGE;
     static constexpr int CA = 2 * DL;                 // 16-byte chunks per A row per stage
     static constexpr int NXC = (BM * CA + kThreads - 1) / kThreads;      // A copies per thread
     static constexpr int NV = (DL * BKL * kJT + kThreads - 1) / kThreads;  // values copies per thread
 };
+
+// Fused bias and activation of four consecutive outputs (columns col..col+3).
+// Kept out of line: the epilogue is unrolled over every vector of a tile, and
+// inlining the activations there would bloat the kernel's code.
+__device__ __noinline__ float4 ep_vec4(float4 o, const float *bias, long long col, int act) {
+    float v[4] = {o.x, o.y, o.z, o.w};
+    if (bias) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] += ep_bias(bias, col + e);
+    }
+    if (act) ep_act_array(v, act);
+    return make_float4(v[0], v[1], v[2], v[3]);
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const float *src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
@@ -101,17 +126,17 @@ template <int DL, int WM, int WK, int TN, bool VT>
 __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p) {
     using TL = Tile32<DL, WM, WK, TN>;
     constexpr int BM = TL::BM, BKL = TL::BKL;
+    using LN = typename TL::LN;
     extern __shared__ __align__(16) float smem[];
     constexpr int kNS = TL::NS;
-    float *sEpi = smem + kNS * TL::STAGE;
     const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(smem);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int w_l = warp / (WM * WK);
-    const int w_m = (warp / WK) % WM;
+    const int w_m = warp / WK;
     const int w_k = warp % WK;
-    const int lane_r = lane >> 2, lane_k = lane & 3;
+    // compute roles: lane = (row group, l, k group), k group fastest
+    const int c_kq = lane % LN::KQ, c_l = (lane / LN::KQ) % DL, c_rg = lane / (LN::KQ * DL);
     const int groups_per_i = p.d / DL;
     const int S = p.n_stages;
     const int my_tiles = (p.n_tiles > (int)blockIdx.x) ? (p.n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
@@ -244,16 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
 #pragma unroll
     for (int g = 0; g < kNS - 1; ++g) issue();
 
-    // Accumulator pairs for fma.rn.f32x2.  DL == 1: acc[m][2q + h] holds row
-    // a_row + 8m at k = b_col + 16q + 2h + (0, 1), X broadcast over a k pair.
-    // DL > 1: acc[pr][kk] holds rows a_row + 16pr + (0, 8) at the thread's
-    // kk-th k (b_col + 16(kk/4) + kk%4), the weight broadcast over a row pair.
-    // (Both are 4 x 2 TN fp32 sums; which one runs faster depends on DL.)
-    constexpr bool kPairK = (DL == 1);
+    // acc[m][2q + h]: row a_row + RG*m, k = b_col + 4*KQ*q + 2h + (0, 1), l = l0 + c_l
     float2 acc[8][TN / 2];
     int buf = 0;  // ring buffer of the stage being computed
-    const int a_row = w_m * 64 + lane_r;                        // thread rows a_row + 8 m
-    const int b_col = w_k * (4 * TN) + lane_k * 4;               // thread k: b_col + 16 q + e
+    const int a_row = w_m * (8 * LN::RG) + c_rg;
+    const int b_col = w_k * TL::KW + 4 * c_kq;
     for (int it = 0; it < my_tiles; ++it) {
         const int tile = (int)blockIdx.x + it * (int)gridDim.x;
 #pragma unroll
@@ -267,98 +287,86 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
             issue();  // into the buffer computed one step ago
             const float *stage = smem + buf * TL::STAGE;
             buf = (buf + 1 == kNS) ? 0 : buf + 1;
-            const float *As = stage + a_row * TL::RA + w_l;
-            const float *Bs = stage + TL::A_WORDS + w_l * TL::PSB + b_col;
+            const float *As = stage + a_row * TL::RA + c_l;
+            const float *Bs = stage + TL::A_WORDS + c_l * TL::PSB + b_col;
 #pragma unroll
             for (int jj = 0; jj < kJT; ++jj) {
                 float am[8];
 #pragma unroll
-                for (int m = 0; m < 8; ++m) am[m] = As[m * 8 * TL::RA + jj * DL];
+                for (int m = 0; m < 8; ++m) am[m] = As[m * LN::RG * TL::RA + jj * DL];
                 float4 bq[TN / 4];
 #pragma unroll
-                for (int q = 0; q < TN / 4; ++q) bq[q] = *reinterpret_cast<const float4 *>(Bs + jj * TL::BKP + 16 * q);
-                if constexpr (kPairK) {
+                for (int q = 0; q < TN / 4; ++q)
+                    bq[q] = *reinterpret_cast<const float4 *>(Bs + jj * TL::BKP + 4 * LN::KQ * q);
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const float2 a2 = make_float2(am[m], am[m]);
+                for (int m = 0; m < 8; ++m) {
+                    const float2 a2 = make_float2(am[m], am[m]);
 #pragma unroll
-                        for (int q = 0; q < TN / 4; ++q) {
-                            acc[m][2 * q] = __ffma2_rn(a2, make_float2(bq[q].x, bq[q].y), acc[m][2 * q]);
-                            acc[m][2 * q + 1] = __ffma2_rn(a2, make_float2(bq[q].z, bq[q].w), acc[m][2 * q + 1]);
-                        }
-                    }
-                } else {
-                    // acc viewed as [4][TN]: acc[pr][kk] at flat index pr * TN + kk
-                    float2 *ac = &acc[0][0];
-#pragma unroll
-                    for (int pr = 0; pr < 4; ++pr) {
-                        const float2 ap = make_float2(am[2 * pr], am[2 * pr + 1]);
-#pragma unroll
-                        for (int q = 0; q < TN / 4; ++q) {
-                            float2 *r = ac + pr * TN + 4 * q;
-                            r[0] = __ffma2_rn(ap, make_float2(bq[q].x, bq[q].x), r[0]);
-                            r[1] = __ffma2_rn(ap, make_float2(bq[q].y, bq[q].y), r[1]);
-                            r[2] = __ffma2_rn(ap, make_float2(bq[q].z, bq[q].z), r[2]);
-                            r[3] = __ffma2_rn(ap, make_float2(bq[q].w, bq[q].w), r[3]);
-                        }
+                    for (int q = 0; q < TN / 4; ++q) {
+                        acc[m][2 * q] = __ffma2_rn(a2, make_float2(bq[q].x, bq[q].y), acc[m][2 * q]);
+                        acc[m][2 * q + 1] = __ffma2_rn(a2, make_float2(bq[q].z, bq[q].w), acc[m][2 * q + 1]);
                     }
                 }
             }
         }
 
-        // Epilogue through its own shared region (the next tile's first stages
-        // are already in flight): Cs[row][l][k], then 16-byte stores of Y.
+        // Epilogue straight from registers.  A thread holds, per row m and k group q,
+        // four consecutive k of its one l.  Shuffles among the lanes of a row group
+        // turn that into four consecutive outputs of Y (DL >= 4: 4x4 transpose over
+        // four l lanes -> (one k, four l); DL = 2: exchange between the two l lanes
+        // -> (two k, two l); DL = 1: already four k), which leave as one 16-byte
+        // store: no shared-memory interleave, no barrier.  The shuffles run on all
+        // lanes; only the stores are predicated.
         const int kb = tile % p.n_kb;
         const int rest = tile / p.n_kb;
         const int gg = rest % p.n_g;
         const long long n0 = (long long)(rest / p.n_g) * BM;
         const int i = gg / groups_per_i, l0 = (gg % groups_per_i) * DL;
-        const int k0 = kb * BKL;
-        constexpr int NP = TL::NP, MP = 8 / NP, RW = 64 / NP;  // rows per warp and pass
+        const int kt = kb * BKL + b_col;  // the thread's first k
+        // output column of the thread's vector for k group q: k_v(q) * d + l_v
+        const int r4 = c_l & 3;
+        const int l_v = DL >= 4 ? l0 + (c_l & ~3) : l0;
+        const int k_off = DL >= 4 ? r4 : DL == 2 ? 2 * c_l : 0;
+        const long long colbase = (long long)i * p.b * p.d + l_v;
 #pragma unroll
-        for (int h = 0; h < NP; ++h) {
+        for (int m = 0; m < 8; ++m) {
+            const long long row = n0 + a_row + LN::RG * m;
+            float *yrow = p.Y + row * p.out_f + colbase;
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm) {
-                const int m = h * MP + mm;
-                float *dst = sEpi + (w_m * RW + lane_r + 8 * mm) * TL::RS + w_l * TL::BKP + b_col;
+            for (int q = 0; q < TN / 4; ++q) {
+                float v[4] = {acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y};
+                if constexpr (DL >= 4) {
+                    // v[e] = (k + e, l = r4) over lanes r4 = 0..3  ->  v[e] = (k + r4, l = e)
 #pragma unroll
-                for (int q = 0; q < TN / 4; ++q) {
-                    float4 o;
-                    if constexpr (kPairK) {
-                        o = make_float4(acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y);
-                    } else {
-                        const float2 *r = &acc[0][0] + (m / 2) * TN + 4 * q;
-                        o = (m % 2 == 0) ? make_float4(r[0].x, r[1].x, r[2].x, r[3].x)
-                                         : make_float4(r[0].y, r[1].y, r[2].y, r[3].y);
+                    for (int t = 0; t < 2; ++t) {
+                        const float snd = (r4 & 1) ? v[2 * t] : v[2 * t + 1];
+                        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+                        if (r4 & 1) v[2 * t] = rcv; else v[2 * t + 1] = rcv;
                     }
-                    *reinterpret_cast<float4 *>(dst + 16 * q) = o;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const float snd = (r4 & 2) ? v[t] : v[t + 2];
+                        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+                        if (r4 & 2) v[t] = rcv; else v[t + 2] = rcv;
+                    }
+                } else if constexpr (DL == 2) {
+                    // lanes l = 0, 1 (lane bit 1): l = 0 takes (k, k+1) x (l0, l1), l = 1 takes (k+2, k+3)
+                    const float s0 = c_l ? v[0] : v[2], s1 = c_l ? v[1] : v[3];
+                    const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+                    const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+                    if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
+                    else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
+                }
+                const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
+                if (row < p.N && k < p.b) {
+                    const long long off = (long long)k * p.d;
+                    float4 o = make_float4(v[0], v[1], v[2], v[3]);
+                    // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
+                    // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
+                    if (p.bias || p.act) o = ep_vec4(o, p.bias, colbase + off, p.act);
+                    *reinterpret_cast<float4 *>(yrow + off) = o;
                 }
             }
-            __syncthreads();
-            constexpr int UO = BKL * DL / 4;  // 16-byte output units per row
-            for (int idx = tid; idx < BM / NP * UO; idx += kThreads) {
-                const int rr = idx / UO;
-                const int uo = idx - rr * UO;
-                const long long row = n0 + (rr / RW) * 64 + h * RW + rr % RW;
-                const int f = uo * 4;  // flat (k_local, l_local)
-                const int kl = f / DL, ll = f % DL;
-                if (row < p.N && k0 + kl < p.b) {
-                    float v[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int fe = f + e;
-                        v[e] = sEpi[rr * TL::RS + (fe % DL) * TL::BKP + fe / DL];
-                    }
-                    const long long col = (long long)i * p.b * p.d + (long long)(k0 + kl) * p.d + l0 + ll;
-                    if (p.bias) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) v[e] += ep_bias(p.bias, col + e);
-                    }
-                    if (p.act) ep_act_array(v, p.act);
-                    *reinterpret_cast<float4 *>(p.Y + row * p.out_f + col) = make_float4(v[0], v[1], v[2], v[3]);
-                }
-            }
-            __syncthreads();
         }
     }
     cp_async_wait<0>();  // no copy may still be landing when the CTA exits
@@ -399,25 +407,59 @@ cudaError_t launch_cfg32(const Problem &pr, const float *vt) {
 
 namespace {
 
+// Tiles of this kernel (dl, wm, wk, tn): BM = 8*RG*wm rows, BKL = KQ*tn*wk k.
+constexpr FmaConfig kFma32Configs[] = {
+    {8, 2, 4, 16}, {8, 4, 2, 16}, {8, 2, 4, 12}, {8, 4, 2, 12},  // 64x64 128x32 64x48 128x24
+    {4, 2, 4, 16}, {4, 1, 8, 16}, {4, 4, 2, 16}, {4, 2, 4, 12}, {4, 1, 8, 12},  // 128x64 64x128 256x32 128x48 64x96
+    {2, 2, 4, 16}, {2, 4, 2, 16}, {2, 8, 1, 16}, {2, 2, 4, 12}, {2, 4, 2, 12},  // 128x128 256x64 512x32 128x96 256x48
+    {1, 4, 2, 16}, {1, 8, 1, 16}, {1, 2, 4, 16}, {1, 4, 2, 12}, {1, 8, 1, 12},  // 256x128 512x64 128x256 256x96 512x48
+};
+
+int cfg_bm(const FmaConfig &c) { return 8 * (32 / (c.dl * (c.dl == 2 ? 2 : c.dl == 1 ? 4 : 1))) * c.wm; }
+int cfg_bk(const FmaConfig &c) { return (c.dl == 2 ? 2 : c.dl == 1 ? 4 : 1) * c.tn * c.wk; }
+
+// Tile choice: the staged-operand reuse BM*BKL/(BM+BKL) per element, discounted
+// by the rows and k a partial tile wastes and by SMs left without a tile.
+FmaConfig fma32_choose(const Problem &p, int dl) {
+    FmaConfig best = {0, 0, 0, 0};
+    double best_score = -1.0;
+    for (const FmaConfig &c : kFma32Configs) {
+        if (c.dl != dl) continue;
+        const int bm = cfg_bm(c), bkl = cfg_bk(c);
+        const double kb = (double)((p.b + bkl - 1) / bkl);
+        const double waste_k = kb * bkl / (double)p.b;
+        const double rb = (double)((p.batch + bm - 1) / bm);
+        const double waste_n = rb * bm / (double)p.batch;
+        const double reuse = (double)bm * bkl / (bm + bkl);
+        const double tiles = rb * kb * (double)(p.a * (p.d / dl));
+        const double fill = std::min(1.0, tiles / (double)sm_count());
+        const double score = reuse * fill / (waste_k * waste_n);
+        if (score > best_score) { best_score = score; best = c; }
+    }
+    return best;
+}
+
 cudaError_t launch_cfg_any(const Problem &p, const FmaConfig &c, const float *vt) {
 #define KS_FMA32_CASE(DL_, WM_, WK_, TN_) \
     if (c.dl == DL_ && c.wm == WM_ && c.wk == WK_ && c.tn == TN_) return launch_cfg32<DL_, WM_, WK_, TN_>(p, vt);
-    KS_FMA32_CASE(8, 1, 1, 16)
-    KS_FMA32_CASE(8, 1, 1, 12)
-    KS_FMA32_CASE(8, 1, 1, 8)
-    KS_FMA32_CASE(4, 2, 1, 16)
-    KS_FMA32_CASE(4, 2, 1, 12)
-    KS_FMA32_CASE(4, 1, 2, 16)
-    KS_FMA32_CASE(4, 1, 2, 12)
-    KS_FMA32_CASE(2, 2, 2, 16)
-    KS_FMA32_CASE(2, 2, 2, 12)
-    KS_FMA32_CASE(2, 4, 1, 16)
-    KS_FMA32_CASE(2, 4, 1, 12)
-    KS_FMA32_CASE(1, 2, 4, 16)
-    KS_FMA32_CASE(1, 2, 4, 12)
+    KS_FMA32_CASE(8, 2, 4, 16)
+    KS_FMA32_CASE(8, 4, 2, 16)
+    KS_FMA32_CASE(8, 2, 4, 12)
+    KS_FMA32_CASE(8, 4, 2, 12)
+    KS_FMA32_CASE(4, 2, 4, 16)
+    KS_FMA32_CASE(4, 1, 8, 16)
+    KS_FMA32_CASE(4, 4, 2, 16)
+    KS_FMA32_CASE(4, 2, 4, 12)
+    KS_FMA32_CASE(4, 1, 8, 12)
+    KS_FMA32_CASE(2, 2, 4, 16)
+    KS_FMA32_CASE(2, 4, 2, 16)
+    KS_FMA32_CASE(2, 8, 1, 16)
+    KS_FMA32_CASE(2, 2, 4, 12)
+    KS_FMA32_CASE(2, 4, 2, 12)
     KS_FMA32_CASE(1, 4, 2, 16)
-    KS_FMA32_CASE(1, 4, 2, 12)
     KS_FMA32_CASE(1, 8, 1, 16)
+    KS_FMA32_CASE(1, 2, 4, 16)
+    KS_FMA32_CASE(1, 4, 2, 12)
     KS_FMA32_CASE(1, 8, 1, 12)
 #undef KS_FMA32_CASE
     return cudaErrorInvalidConfiguration;
@@ -433,7 +475,10 @@ cudaError_t launch_cfg_any(const Problem &p, const FmaConfig &c, const float *vt
 // in-place path on the fp32 sweep: 1.20x median for d % 8 == 0; for smaller
 // l widths the gain (1.01-1.03x) did not cover the transpose on mid-size runs.
 // If the workspace cannot be had, the values are read in place.
-cudaError_t launch_fma32(const Problem &p, const FmaConfig &c) {
+cudaError_t launch_fma32(const Problem &p, const FmaConfig &c_in) {
+    // the l width comes from the caller's plan, the tile from this kernel's table
+    const FmaConfig c = fma32_choose(p, c_in.dl);
+    if (c.dl == 0) return cudaErrorInvalidConfiguration;
     const long long nvals = p.a * p.b * p.c * p.d;
     const double flops = 2.0 * (double)p.batch * (double)nvals;
     if (c.dl == 8 && p.b % 4 == 0 && flops >= 1073741824.0 && nvals * 4 <= (64LL << 20)) {
