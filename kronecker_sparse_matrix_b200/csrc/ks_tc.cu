@@ -258,6 +258,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ in-place transpose (DLS > 1)
         if (DLS > 1) {
             const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
+            // task -> (16-byte unit q of a raw row, row group g8).  16-byte shared
+            // accesses are served eight lanes at a time, so every eight
+            // consecutive lanes must reach eight distinct bank groups, both when
+            // reading the raw chunk (group = q) and when writing the padded planes
+            // (group = g8 + the unit's j mod 8); for two and four l the row group
+            // is skewed by the unit for that.
+            auto task_unit = [&](int task, int &q, int &g8) {
+                if (DLS == 8) {
+                    q = task % UNITS;
+                    g8 = task / UNITS;
+                } else {
+                    q = task & 7;
+                    g8 = ((task >> 3) + (q >> (DLS == 2 ? 1 : 2))) & 15;
+                }
+            };
             uint32_t xq = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
@@ -271,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint4 out[TASKS][8];
 #pragma unroll
                         for (int k = 0; k < TASKS; ++k) {
-                            const int task = t + 128 * k;
-                            const int q = task % UNITS, g8 = task / UNITS;
+                            int q, g8;
+                            task_unit(t + 128 * k, q, g8);
                             uint4 in[8];
 #pragma unroll
                             for (int r = 0; r < 8; ++r)
@@ -282,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bar_sync(1, 128);  // every read of the raw chunk is done
 #pragma unroll
                         for (int k = 0; k < TASKS; ++k) {
-                            const int task = t + 128 * k;
-                            const int q = task % UNITS, g8 = task / UNITS;
+                            int q, g8;
+                            task_unit(t + 128 * k, q, g8);
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
                                 const int f = 8 * q + e;
