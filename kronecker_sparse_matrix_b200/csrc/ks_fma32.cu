@@ -328,43 +328,88 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
         const int l_v = DL >= 4 ? l0 + (c_l & ~3) : l0;
         const int k_off = DL >= 4 ? r4 : DL == 2 ? 2 * c_l : 0;
         const long long colbase = (long long)i * p.b * p.d + l_v;
+        // Two copies of the unrolled store loop: the plain one carries no call
+        // site at all (the fused bias/activation's call, even when skipped, made
+        // the plain loop slower), the fused one calls the out-of-line helper.
+        if (p.bias == nullptr && p.act == 0) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const long long row = n0 + a_row + LN::RG * m;
-            float *yrow = p.Y + row * p.out_f + colbase;
+            for (int m = 0; m < 8; ++m) {
+                const long long row = n0 + a_row + LN::RG * m;
+                float *yrow = p.Y + row * p.out_f + colbase;
 #pragma unroll
-            for (int q = 0; q < TN / 4; ++q) {
-                float v[4] = {acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y};
-                if constexpr (DL >= 4) {
-                    // v[e] = (k + e, l = r4) over lanes r4 = 0..3  ->  v[e] = (k + r4, l = e)
+                for (int q = 0; q < TN / 4; ++q) {
+                    float v[4] = {acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y};
+                    if constexpr (DL >= 4) {
+                        // v[e] = (k + e, l = r4) over lanes r4 = 0..3  ->  v[e] = (k + r4, l = e)
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const float snd = (r4 & 1) ? v[2 * t] : v[2 * t + 1];
-                        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
-                        if (r4 & 1) v[2 * t] = rcv; else v[2 * t + 1] = rcv;
+                        for (int t = 0; t < 2; ++t) {
+                            const float snd = (r4 & 1) ? v[2 * t] : v[2 * t + 1];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+                            if (r4 & 1) v[2 * t] = rcv; else v[2 * t + 1] = rcv;
+                        }
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const float snd = (r4 & 2) ? v[t] : v[t + 2];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+                            if (r4 & 2) v[t] = rcv; else v[t + 2] = rcv;
+                        }
+                    } else if constexpr (DL == 2) {
+                        // lanes l = 0, 1 (lane bit 1): l = 0 takes (k, k+1) x (l0, l1), l = 1 takes (k+2, k+3)
+                        const float s0 = c_l ? v[0] : v[2], s1 = c_l ? v[1] : v[3];
+                        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+                        const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+                        if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
+                        else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
                     }
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const float snd = (r4 & 2) ? v[t] : v[t + 2];
-                        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
-                        if (r4 & 2) v[t] = rcv; else v[t + 2] = rcv;
+                    const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
+                    if (row < p.N && k < p.b) {
+                        const long long off = (long long)k * p.d;
+                        float4 o = make_float4(v[0], v[1], v[2], v[3]);
+                        // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
+                        // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
+                        *reinterpret_cast<float4 *>(yrow + off) = o;
                     }
-                } else if constexpr (DL == 2) {
-                    // lanes l = 0, 1 (lane bit 1): l = 0 takes (k, k+1) x (l0, l1), l = 1 takes (k+2, k+3)
-                    const float s0 = c_l ? v[0] : v[2], s1 = c_l ? v[1] : v[3];
-                    const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
-                    const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
-                    if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
-                    else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
                 }
-                const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
-                if (row < p.N && k < p.b) {
-                    const long long off = (long long)k * p.d;
-                    float4 o = make_float4(v[0], v[1], v[2], v[3]);
-                    // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
-                    // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
-                    if (p.bias || p.act) o = ep_vec4(o, p.bias, colbase + off, p.act);
-                    *reinterpret_cast<float4 *>(yrow + off) = o;
+            }
+        } else {
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const long long row = n0 + a_row + LN::RG * m;
+                float *yrow = p.Y + row * p.out_f + colbase;
+#pragma unroll
+                for (int q = 0; q < TN / 4; ++q) {
+                    float v[4] = {acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y};
+                    if constexpr (DL >= 4) {
+                        // v[e] = (k + e, l = r4) over lanes r4 = 0..3  ->  v[e] = (k + r4, l = e)
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const float snd = (r4 & 1) ? v[2 * t] : v[2 * t + 1];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+                            if (r4 & 1) v[2 * t] = rcv; else v[2 * t + 1] = rcv;
+                        }
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const float snd = (r4 & 2) ? v[t] : v[t + 2];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+                            if (r4 & 2) v[t] = rcv; else v[t + 2] = rcv;
+                        }
+                    } else if constexpr (DL == 2) {
+                        // lanes l = 0, 1 (lane bit 1): l = 0 takes (k, k+1) x (l0, l1), l = 1 takes (k+2, k+3)
+                        const float s0 = c_l ? v[0] : v[2], s1 = c_l ? v[1] : v[3];
+                        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+                        const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+                        if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
+                        else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
+                    }
+                    const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
+                    if (row < p.N && k < p.b) {
+                        const long long off = (long long)k * p.d;
+                        float4 o = make_float4(v[0], v[1], v[2], v[3]);
+                        // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
+                        // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
+                        o = ep_vec4(o, p.bias, colbase + off, p.act);
+                        *reinterpret_cast<float4 *>(yrow + off) = o;
+                    }
                 }
             }
         }
