@@ -20,17 +20,23 @@
 //   warp 0      TMA producer: raw X chunks (128 rows x 64..128 (j, l)
 //               elements; l innermost, the only shape a tensor map can fetch
 //               from the strided layout) into the ring, and the values of
-//               the same j range (K-major core matrices) into a 3..4-deep ring;
+//               the same j range into a 3..4-deep ring, as DLS K-major planes
+//               whose rows (one k, the chunk's j) carry the swizzle of their
+//               width (a TMA copy moves about one box row per clock, so the
+//               rows are made as wide as the chunk allows);
 //   warps 2..5  (DLS > 1) transpose each chunk in place, in registers, from
-//               [row][j][l] to one MN-major no-swizzle operand plane per l;
-//               for d = 1 the TMA box already lands as the 128-byte-swizzled
-//               K-major tile the MMA reads, and these warps idle;
+//               [row][j][l] to one MN-major no-swizzle operand plane per l,
+//               row groups padded and skewed so every quarter-warp's 16-byte
+//               accesses reach eight bank groups; for d = 1 the TMA box
+//               already lands as the 128-byte-swizzled K-major tile the MMA
+//               reads, and these warps idle;
 //   warp 1      one thread issues tcgen05.mma (kind::f16, M=128, N=bp, K=16)
 //               per plane and K step, commits to mbarriers;
 //   warps 6..9  tcgen05.ld the accumulators (each warp its 32 TMEM lanes =
 //               rows), round to bf16, interleave the l planes back into Y's
-//               (k, l) order in a swizzled shared-memory staging box, and
-//               copy it to Y in whole 128-byte row segments.
+//               (k, l) order in a shared-memory staging box of 32 rows, and
+//               hand it to a TMA tensor store when the box is contiguous in Y
+//               (d == DLS), or copy it out in 16-byte stores otherwise.
 //
 // Every mbarrier wait is bounded (about one second of %globaltimer); a wait
 // that runs out sets the device status word and raises the CTA's abort flag,
