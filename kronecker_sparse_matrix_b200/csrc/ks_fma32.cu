@@ -81,7 +81,10 @@ struct Tile32 {
     // plane stride: PSB/4 odd (DL = 8, 4) or = 2 (mod 8) (DL = 2, with the k pair of lanes)
     static constexpr int PSB = kJT * BKP + (DL == 2 ? 8 : 4);
     static constexpr int STAGE = A_WORDS + DL * PSB;  // words
-    static constexpr int NS = (4 * STAGE * 4 <= 232448) ? 4 : 3;
+    // ring depth: 4 stages for DL = 4, 3 otherwise (measured: a fourth stage
+    // helps DL = 4; for the other widths the larger shared-memory carve-out
+    // leaves less L1 for the 4-byte values copies, 1-2% slower)
+    static constexpr int NS = (DL == 4 && 4 * STAGE * 4 <= 232448) ? 4 : 3;
     static constexpr int SMEM_FLOATS = NS * STAGE;
     static constexpr int CA = 2 * DL;                 // 16-byte chunks per A row per stage
     static constexpr int NXC = (BM * CA + kThreads - 1) / kThreads;      // A copies per thread
