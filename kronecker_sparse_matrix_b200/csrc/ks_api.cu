@@ -86,7 +86,7 @@ ks_status make_problem(const void *X, const void *V, int64_t a, int64_t b, int64
                        int64_t batch, void *Y, int dtype, void *stream, Problem *p, bool *noop) {
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
-    int64_t in_f, out_f, nvals;
+    int64_t in_f = 0, out_f = 0, nvals = 0;
     if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
     *noop = (batch == 0);
     if (*noop) return KS_OK;
@@ -237,7 +237,7 @@ ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch, int
     if (!variant) return fail(KS_ERR_INVALID_ARG, "variant must be non-null");
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
-    int64_t in_f, out_f, nvals;
+    int64_t in_f = 0, out_f = 0, nvals = 0;
     if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
     // Assume 256-byte aligned buffers, as a fresh allocation has.
     static const char dummy[16] __attribute__((aligned(256))) = {};
@@ -274,7 +274,7 @@ ks_status ks_chain_ep(const void *X, const void *const *factors, const ks_patter
     int64_t widest = 0;
     for (int t = 0; t < n_factors; ++t) {
         const ks_pattern &q = patterns[t];
-        int64_t in_f, out_f, nvals;
+        int64_t in_f = 0, out_f = 0, nvals = 0;
         if ((s = check_sizes(q.a, q.b, q.c, q.d, batch, &in_f, &out_f, &nvals)) != KS_OK) {
             char tmp[512];
             snprintf(tmp, sizeof(tmp), "factor %d: %s", t, g_msg);
@@ -360,7 +360,7 @@ ks_status ks_matmul_dx(const void *dY, const void *values, int64_t a, int64_t b,
                        int64_t batch, void *dX, int dtype, void *stream) {
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
-    int64_t in_f, out_f, nvals;
+    int64_t in_f = 0, out_f = 0, nvals = 0;
     if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
     if (batch == 0) return KS_OK;
     if (!dY || !values || !dX) return fail(KS_ERR_INVALID_ARG, "dY, values and dX must be non-null");
@@ -406,7 +406,7 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int6
                        void *dV, int dtype, void *stream) {
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;
-    int64_t in_f, out_f, nvals;
+    int64_t in_f = 0, out_f = 0, nvals = 0;
     if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
     if (!dV) return fail(KS_ERR_INVALID_ARG, "dV must be non-null");
     const int elem = dtype == KS_BF16 ? 2 : 4;
