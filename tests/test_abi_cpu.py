@@ -99,6 +99,21 @@ def test_chain_validation(lib):
     assert lib.ks_chain(P, ptrs, ok, 2, 0, P * 8, 0, None) == 0  # batch 0: no-op
 
 
+def test_noalloc_chain_validates_on_the_host(lib):
+    # the fixed scratch holds 16 MiB per intermediate: a 4096-wide fp32 intermediate fits
+    # 1024 rows, and 1025 are refused before any device call
+    pats = (_lib.KsPattern * 2)(_lib.KsPattern(1, 4096, 4096, 1), _lib.KsPattern(1, 4096, 4096, 1))
+    ptrs = (ctypes.c_void_p * 2)(P, P)
+    assert lib.ks_chain_noalloc(P, ptrs, pats, 2, 1025, P * 8, 0, None) == 1
+    assert b"exceeds the fixed scratch" in lib.ks_last_error()
+    bad = (_lib.KsPattern * 2)(_lib.KsPattern(1, 2, 2, 2), _lib.KsPattern(1, 2, 2, 1))
+    assert lib.ks_chain_noalloc(P, ptrs, bad, 2, 4, P * 8, 0, None) == 1
+    assert b"input width" in lib.ks_last_error()
+    assert lib.ks_chain_noalloc(P, ptrs, pats, 2, 4, P * 8, 7, None) == 1  # unknown dtype
+    assert lib.ks_chain_noalloc(P, (ctypes.c_void_p * 2)(P, None), pats, 2, 4, P * 8, 0, None) == 1
+    assert lib.ks_chain_noalloc(P, ptrs, pats, 2, 0, P * 8, 0, None) == 0  # batch 0: no-op
+
+
 def test_plan_is_host_only_and_sensible(lib):
     v = ctypes.c_int(-1)
     assert lib.ks_plan(1, 192, 48, 8, 25216, 0, ctypes.byref(v)) == 0
