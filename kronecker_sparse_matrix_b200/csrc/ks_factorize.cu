@@ -1,5 +1,5 @@
-// Hierarchical butterfly factorization on the GPU (mlsanity.com page on
-// butterfly factorization, abstract: a matrix is split recursively into two
+// Hierarchical butterfly factorization on the GPU (taxoreview.com page, third
+// abstract: a matrix is split recursively into two
 // factors with butterfly supports, each split a two-factor fixed-support
 // factorization with exact recovery).
 //

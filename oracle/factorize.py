@@ -2,8 +2,8 @@
 ONLY: imported by tests, the smoke check and the benchmark's CPU legs, never
 by the product path).
 
-What it follows: the mlsanity.com page on butterfly factorization (its
-abstract): a matrix is factored into sparse factors with butterfly supports
+What it follows: the taxoreview.com page's third abstract (hierarchical
+butterfly factorization): a matrix is factored into sparse factors with butterfly supports
 by recursively splitting it into two factors, each split a two-factor
 fixed-support factorization, with exact recovery when the matrix is such a
 product.  The page gives no formulas; the steps below are the plain reading

@@ -47,3 +47,14 @@ def test_epilogue_is_product_plus_bias_then_activation(act):
     Z = oracle.matmul(X, V, p) + bias[None, :]
     np.testing.assert_allclose(oracle.matmul_epilogue(X, V, p, bias, act), oracle.activation(Z, act), rtol=0, atol=0)
     np.testing.assert_allclose(oracle.matmul_epilogue(X, V, p, None, "none"), oracle.matmul(X, V, p), rtol=0, atol=0)
+
+
+def test_epilogue_matches_hand_worked_examples():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "epilogue_examples.json")
+    for case in json.load(open(path))["cases"]:
+        p = tuple(case["pattern"])
+        got = oracle.matmul_epilogue(np.array(case["X"], dtype=float), np.array(case["values"], dtype=float), p,
+                                     np.array(case["bias"], dtype=float), case["act"])
+        np.testing.assert_array_equal(got, np.array(case["Y"], dtype=float), err_msg=case["name"])
