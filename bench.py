@@ -11,10 +11,12 @@ stream).
 
 Per run r: FLOPs_r = 2*N*a*b*c*d, bytes_r = s*(N*a*c*d + N*a*b*d + a*b*c*d),
 roofline_r = min(P_peak, BW * FLOPs_r / bytes_r) with BW the measured HBM copy
-bandwidth, P_peak the fp32 FMA peak (148 SMs x 128 lanes x 2 x 1965 MHz) for
-fp32 runs and the measured bf16 tensor peak for bf16 runs;
-frac_r = (FLOPs_r / t_r) / roofline_r.  ``value`` is the median of frac_r over
-the runs.  One JSON line is printed (rank 0).
+bandwidth and P_peak the fp32 FMA peak for fp32 runs (measured in the same run
+by the library's FMA-rate probe; 148 SMs x 128 lanes x 2 x 1965 MHz = 74.45
+TFLOP/s derived, as a note), the TF32 tensor peak for TF32 runs (a torch
+TF32 matmul timed in the same run) and the measured bf16 tensor peak for bf16
+runs; frac_r = (FLOPs_r / t_r) / roofline_r.  ``value`` is the median of frac_r
+over the runs.  One JSON line is printed (rank 0).
 
 ``--impl reference`` times the CPU oracle (the plain C loops under oracle/)
 on a bounded sample of the same workload, in the same unit.
@@ -39,7 +41,7 @@ import torch  # noqa: E402
 
 from kronecker_sparse_matrix_b200 import inputs  # noqa: E402
 
-FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12  # 74.45: SMs x FP32 lanes x 2 flop x max SM clock
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12  # 74.45: SMs x FP32 lanes x 2 flop x max SM clock (derived)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "KS matmul GFLOP/s and HBM GB/s at 1 B200 as fraction of roofline, pattern median"
 L2_FLUSH_BYTES = 256 * 1024 * 1024
@@ -81,11 +83,61 @@ def launches_per_call(p, n, dtype, variant):
     return 1
 
 
+def elem_bytes(dtype):
+    return 2 if dtype == "bf16" else 4
+
+
 def roofline_tflops(p, n, dtype, peaks):
-    s = 4 if dtype == "fp32" else 2
-    ai = run_flops(p, n) / run_bytes(p, n, s)
-    p_peak = FP32_FMA_PEAK_TFLOPS if dtype in ("fp32", "tf32") else peaks["bf16_tflops"]
+    ai = run_flops(p, n) / run_bytes(p, n, elem_bytes(dtype))
+    p_peak = {"fp32": peaks.get("fp32_fma_tflops", FP32_FMA_PEAK_TFLOPS),
+              "tf32": peaks.get("tf32_tflops", peaks["bf16_tflops"] / 2),
+              "bf16": peaks["bf16_tflops"]}[dtype]
     return min(p_peak, peaks["hbm_gbs"] * ai / 1e3)
+
+
+def measure_fma_peak(dev, reps=5):
+    """TFLOP/s of the library's FP32 FMA-rate probe (best of `reps` launches of
+    about 3 ms, 4 blocks of 256 threads per SM), timed with CUDA events."""
+    from kronecker_sparse_matrix_b200 import _lib
+    lib = _lib.load()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks, iters = 4 * sms, 40000
+    out = torch.empty(blocks, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    best = float("inf")
+    for r in range(reps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _lib.check(lib.ks_fma_rate_probe(out.data_ptr(), blocks, iters, stream.cuda_stream))
+        e1.record(stream)
+        e1.synchronize()
+        if r >= 2:
+            best = min(best, e0.elapsed_time(e1) / 1e3)
+    return blocks * 256 * iters * 32 / best / 1e12
+
+
+def measure_tf32_peak(dev, n=8192, reps=5):
+    """TFLOP/s of a torch (cuBLAS) fp32 matmul n^3 with TF32 tensor cores
+    allowed, best of `reps`."""
+    a = torch.randn(n, n, device=dev)
+    b = torch.randn(n, n, device=dev)
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        stream = torch.cuda.current_stream(dev)
+        best = float("inf")
+        for r in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch.matmul(a, b)
+            e1.record(stream)
+            e1.synchronize()
+            if r >= 2:
+                best = min(best, e0.elapsed_time(e1) / 1e3)
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    del a, b
+    return 2.0 * n ** 3 / best / 1e12
 
 
 # ---------------------------------------------------------------------------- workloads
@@ -98,6 +150,8 @@ def workload_runs(name):
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "fp32", i) for i, p in enumerate(inputs.sweep_patterns())]
     if name == "sweep-bf16":
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "bf16", i) for i, p in enumerate(inputs.sweep_patterns())]
+    if name == "sweep-tf32":
+        return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "tf32", i) for i, p in enumerate(inputs.sweep_patterns())]
     if name == "sweep-quick":  # every 8th pattern, for development only
         pats = inputs.sweep_patterns()
         return [(f"sweep[{i}]", pats[i], inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16")
@@ -124,6 +178,10 @@ WORKLOAD_TEXT = {
 
 def torch_dtype(dt):
     return torch.float32 if dt in ("fp32", "tf32") else torch.bfloat16
+
+
+def is_tf32(dt):
+    return dt == "tf32"
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -267,26 +325,33 @@ def gpu_arm(args, rank, world, local):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     results = []
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if args.save_clocks else None
+    clock_path = None
+    if args.save_clocks:
+        clock_path = args.save_clocks if world == 1 else f"{args.save_clocks}.rank{rank}"
 
     # --- device-resident timing ------------------------------------------------
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local, clock_path) as clocks:
+        # the compute peaks of this device, measured in the same run
+        peaks["fp32_fma_tflops"] = measure_fma_peak(dev)
+        peaks["tf32_tflops"] = measure_tf32_peak(dev)
+        torch.cuda.synchronize(dev)
+        barrier(world)
         for label, p, n, dt, seed in runs:
             f = inputs.factor_inputs(p, n, seed=rank_seed(seed, rank), dtype=torch_dtype(dt), device=dev)
             Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
-            variant = ks.plan(p, n, ks.ks_dtype_of(f.X))
+            tf32 = is_tf32(dt)
+            variant = ks.plan(p, n, ks.ks_dtype_of(f.X, tf32))
             for _ in range(args.warmup):
-                ks.matmul(f.X, f.values, p, out=Y)
+                ks.matmul(f.X, f.values, p, out=Y, tf32=tf32)
             times = []
             for _ in range(args.steps):
                 flush.zero_()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                ks.matmul(f.X, f.values, p, out=Y)
+                ks.matmul(f.X, f.values, p, out=Y, tf32=tf32)
                 e1.record(stream)
                 e1.synchronize()
                 times.append(e0.elapsed_time(e1) / 1e3)
@@ -308,7 +373,7 @@ def gpu_arm(args, rank, world, local):
     for r in results:
         p, n, dt = r["pattern"], r["batch"], r["dtype"]
         t = statistics.mean(r["times"])
-        s = 4 if dt == "fp32" else 2
+        s = elem_bytes(dt)
         r["t"] = t
         r["flops"] = run_flops(p, n) * world
         r["bytes"] = run_bytes(p, n, s) * world
@@ -330,8 +395,8 @@ def e2e_measure(args, runs, rank, world, dev, peaks):
     import kronecker_sparse_matrix_b200 as ks
 
     steps = max(1, min(args.steps, args.e2e_steps))
-    max_x = max(n * inputs.in_features(p) * (4 if dt == "fp32" else 2) for _, p, n, dt, _ in runs)
-    max_y = max(n * inputs.out_features(p) * (4 if dt == "fp32" else 2) for _, p, n, dt, _ in runs)
+    max_x = max(n * inputs.in_features(p) * elem_bytes(dt) for _, p, n, dt, _ in runs)
+    max_y = max(n * inputs.out_features(p) * elem_bytes(dt) for _, p, n, dt, _ in runs)
     max_v = max(p[0] * p[1] * p[2] * p[3] * 4 for _, p, _, _, _ in runs)
     hx = torch.empty(max_x, dtype=torch.uint8, pin_memory=True)
     hy = torch.empty(max_y, dtype=torch.uint8, pin_memory=True)
@@ -352,10 +417,11 @@ def e2e_measure(args, runs, rank, world, dev, peaks):
         dX, dV = torch.empty_like(f.X), torch.empty_like(f.values)
         dY = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
         del f
+        tf32 = is_tf32(dt)
         # warm-up once (untimed)
         dX.copy_(hxv, non_blocking=True)
         dV.copy_(hvv, non_blocking=True)
-        ks.matmul(dX, dV, p, out=dY)
+        ks.matmul(dX, dV, p, out=dY, tf32=tf32)
         hyv.copy_(dY, non_blocking=True)
         torch.cuda.synchronize(dev)
         for _ in range(steps):
@@ -364,7 +430,7 @@ def e2e_measure(args, runs, rank, world, dev, peaks):
             e0.record(stream)
             dX.copy_(hxv, non_blocking=True)
             dV.copy_(hvv, non_blocking=True)
-            ks.matmul(dX, dV, p, out=dY)
+            ks.matmul(dX, dV, p, out=dY, tf32=tf32)
             hyv.copy_(dY, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
@@ -474,17 +540,32 @@ def extra_configs(args, dev, peaks):
         return statistics.median(ts)
 
     out = {}
-    for name, dt in [("vit", "fp32"), ("gpt2", "fp32"), ("gpt2", "bf16")]:
+    for name, dt in [("vit", "fp32"), ("vit", "tf32"), ("gpt2", "fp32"), ("gpt2", "tf32"), ("gpt2", "bf16")]:
         f = getattr(inputs, name)(dtype=torch_dtype(dt), device=dev)
         p, n = f.pattern, f.batch
+        tf32 = is_tf32(dt)
         Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
-        t = timed(lambda: ks.matmul(f.X, f.values, p, out=Y), args.steps)
-        s = 4 if dt == "fp32" else 2
+        t = timed(lambda: ks.matmul(f.X, f.values, p, out=Y, tf32=tf32), args.steps)
+        s = elem_bytes(dt)
         tf = run_flops(p, n) / t / 1e12
+        roof = roofline_tflops(p, n, dt, peaks)
+        bound = "hbm" if roof < (peaks["fp32_fma_tflops"] if dt == "fp32" else peaks[f"{dt}_tflops"]) else "compute"
         out[f"{name}-{dt}"] = {"pattern": list(p), "batch": n, "us": t * 1e6, "tflops": tf,
                                "gbs": run_bytes(p, n, s) / t / 1e9,
-                               "frac": tf / roofline_tflops(p, n, dt, peaks),
-                               "variant": ks.plan(p, n, ks.ks_dtype_of(f.X))}
+                               "frac": tf / roof, "bound": bound,
+                               "variant": ks.plan(p, n, ks.ks_dtype_of(f.X, tf32))}
+        del f, Y
+    # the sweep in TF32 (fp32 buffers, tensor cores): median fraction of its roofline
+    tf32_fr = []
+    for label, p, n, dt, seed in workload_runs("sweep-tf32"):
+        f = inputs.factor_inputs(p, n, seed=seed, device=dev)
+        Y = torch.empty((n, inputs.out_features(p)), dtype=f.X.dtype, device=dev)
+        t = timed(lambda: ks.matmul(f.X, f.values, p, out=Y, tf32=True), min(args.steps, 3))
+        tf32_fr.append(run_flops(p, n) / t / 1e12 / roofline_tflops(p, n, "tf32", peaks))
+        del f, Y
+    out["sweep-tf32"] = {"runs": len(tf32_fr), "median_frac": statistics.median(tf32_fr),
+                         "note": "the 258 sweep patterns with fp32 buffers on the TF32 tensor-core path; "
+                                 "roofline min(TF32 peak, HBM x AI), all HBM-bound"}
     # fused epilogue: act(X K^T + bias) with GELU (tanh form), the MLP-up layer
     for name, dt in [("vit", "fp32"), ("gpt2", "bf16")]:
         f = getattr(inputs, name)(dtype=torch_dtype(dt), device=dev)
@@ -522,7 +603,7 @@ def extra_configs(args, dev, peaks):
     del A, c
     for dt in ("fp32", "bf16"):
         c = inputs.butterfly(device=dev, dtype=torch_dtype(dt))
-        s = 4 if dt == "fp32" else 2
+        s = elem_bytes(dt)
         Y = torch.empty_like(c.X)
         vbytes = sum(p[0] * p[1] * p[2] * p[3] for p in c.patterns) * s
         for fused in (True, False):
@@ -552,7 +633,8 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=128)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--save-clocks", action="store_true")
+    ap.add_argument("--save-clocks", default=None, metavar="PATH",
+                    help="also write the nvidia-smi clock samples of the timed region to PATH")
     ap.add_argument("--details", default=None, help="write per-run results as JSON here")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -598,9 +680,12 @@ def main(argv=None):
         dom = fam[dom_key]
         if dom_key.startswith("fma-fp32"):
             achieved = dom["flops"] / dom["t"] / 1e12
-            roof = {"bound": "alu", "achieved": achieved, "peak": FP32_FMA_PEAK_TFLOPS, "unit": "TFLOP/s",
-                    "frac": achieved / FP32_FMA_PEAK_TFLOPS,
-                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"}
+            pk = peaks["fp32_fma_tflops"]
+            roof = {"bound": "alu", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
+                    "peak_source": "measured in this run: the library's FP32 FMA-rate probe (fma.rn.f32x2 chains, "
+                                   "CUDA events); derived 148 SMs x 128 lanes x 2 flop x 1965 MHz = "
+                                   f"{FP32_FMA_PEAK_TFLOPS:.2f} TFLOP/s, frac against it "
+                                   f"{achieved / FP32_FMA_PEAK_TFLOPS:.4f}"}
         elif dom_key.startswith("tc"):
             achieved = dom["bytes"] / dom["t"] / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -636,7 +721,12 @@ def main(argv=None):
                                              for r in results),
             "clocks": clocks,
             "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
-                      "fp32_fma_tflops": FP32_FMA_PEAK_TFLOPS, "source": peaks["source"]},
+                      "fp32_fma_tflops": peaks["fp32_fma_tflops"], "fp32_fma_tflops_derived": FP32_FMA_PEAK_TFLOPS,
+                      "tf32_tflops": peaks["tf32_tflops"],
+                      "fp32_fma_flop_per_sm_clock": (peaks["fp32_fma_tflops"] * 1e12 / 148 /
+                                                     (clocks["sm_mhz"] * 1e6)) if clocks.get("sm_mhz") else None,
+                      "source": f"HBM and bf16: {peaks['source']} (MEASURED_PEAKS.json); FP32 FMA and TF32: "
+                                "measured in this run"},
             "extra": extra,
         }
         if args.details:

@@ -26,8 +26,10 @@
  *     values is the contiguous array values[a][d][b][c].
  *   - X, values and Y share one storage type: fp32 for KS_F32 and KS_TF32,
  *     bf16 for KS_BF16 (Y is written in bf16, rounded to nearest even from an
- *     fp32 accumulator).  KS_TF32 reads fp32 buffers and multiplies in TF32
- *     (accumulating in fp32); it is never chosen silently for KS_F32.
+ *     fp32 accumulator).  KS_TF32 reads and writes fp32 buffers; where the
+ *     tensor-core kernel takes the pattern (see KS_TF32 below) the products
+ *     use TF32 operands with fp32 accumulation, elsewhere they are full fp32.
+ *     TF32 is never chosen silently for KS_F32.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *     call is asynchronous on that stream; the return value reports only
  *     errors found before or at launch.  Errors found on the device (a bounded
@@ -51,10 +53,15 @@ extern "C" {
 #endif
 
 /* Storage / arithmetic type of X, values and Y. */
+/* KS_TF32 and KS_BF16 run on the tcgen05 tensor cores when the pattern fits
+ * the tensor-core kernel: d in {1, 2, 4} or a multiple of 8; c a multiple of
+ * 8 (TF32) or 16 (BF16); b a multiple of 16; b*c > 64; X, values and Y
+ * 16-byte aligned.  Other patterns run on CUDA cores with fp32 arithmetic
+ * (at least the accuracy of the tensor-core path). */
 typedef enum ks_dtype {
-    KS_F32 = 0,  /* fp32 storage, fp32 FMA arithmetic                         */
-    KS_TF32 = 1, /* fp32 storage, TF32 tensor-core products, fp32 accumulate  */
-    KS_BF16 = 2  /* bf16 storage, bf16 tensor-core products, fp32 accumulate  */
+    KS_F32 = 0,  /* fp32 storage, fp32 FMA arithmetic (CUDA cores)                 */
+    KS_TF32 = 1, /* fp32 storage, TF32 tensor-core products, fp32 accumulate       */
+    KS_BF16 = 2  /* bf16 storage, bf16 tensor-core products, fp32 accumulate       */
 } ks_dtype;
 
 typedef enum ks_status {
@@ -62,7 +69,7 @@ typedef enum ks_status {
     KS_ERR_INVALID_ARG = 1, /* bad pattern, batch, dtype, pointer or overlap          */
     KS_ERR_MISALIGNED = 2,  /* pointer not aligned to its element size                */
     KS_ERR_UNSUPPORTED = 3, /* variant forced on a pattern it cannot run              */
-    KS_ERR_ALLOC = 4,       /* workspace allocation failed (ks_chain)                 */
+    KS_ERR_ALLOC = 4,       /* workspace allocation failed                            */
     KS_ERR_CUDA = 5,        /* a CUDA runtime call failed; see ks_last_error()        */
     KS_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (ks_sync_status)    */
 } ks_status;
@@ -95,7 +102,16 @@ typedef struct ks_pattern {
 
 /* Y = X * K^T for one KS factor (see the top of this file for the layout).
  * dtype is a ks_dtype; stream a cudaStream_t.  The pattern heuristic picks the
- * kernel. */
+ * kernel.
+ *
+ * Workspace: for KS_F32 (and KS_TF32 patterns on CUDA cores) with d % 8 == 0,
+ * b % 4 == 0, at least 2^30 flop (2*batch*a*b*c*d) and values of at most
+ * 64 MiB, the product first writes a copy of the values transposed per block
+ * into a stream-ordered workspace (a*b*c*d floats) from the library's memory
+ * pool (see ks_chain) and frees it on the stream after the kernel; if that
+ * allocation fails the values are read in place and the result is the same.
+ * Every other product allocates nothing.  ks_chain_noalloc never takes this
+ * workspace. */
 ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
                     int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
                     void *stream);
@@ -238,6 +254,37 @@ ks_status ks_chain_noalloc(const void *X, const void *const *factors,
  * ordered, freed before return). */
 ks_status ks_butterfly_factorize(const void *A, int log2n, void *const *factors,
                                  int dtype, void *stream);
+
+/* The library's workspace memory (not part of the paper's operation; for
+ * callers that budget device memory).  *allocations (if non-NULL) receives
+ * the number of workspace allocations the library has made from its pools
+ * since the process started, on all devices; *reserved_bytes (if non-NULL)
+ * the device memory the pool of the current device holds now (it keeps freed
+ * workspace for later calls, see ks_chain).  Host-only apart from the pool
+ * query; KS_ERR_CUDA if the current device has no pool. */
+ks_status ks_workspace_info(int64_t *allocations, int64_t *reserved_bytes);
+
+/* Measurement helper (not part of the paper's operation): the FP32 FMA
+ * throughput of the current device's CUDA cores, the peak that bounds the
+ * fp32 products.  Launches `blocks` blocks of 256 threads on `stream`; every
+ * thread issues iters x 8 packed FMAs (fma.rn.f32x2, four flops each), so a
+ * launch is blocks * 256 * iters * 32 flop.  out is a DEVICE array of
+ * `blocks` floats (a checksum per block, so no work is optimised away).
+ * Time it with events on `stream`.  KS_ERR_INVALID_ARG for a null out or
+ * non-positive blocks / iters. */
+ks_status ks_fma_rate_probe(float *out, int blocks, int64_t iters, void *stream);
+
+/* Fault injection for tests (read on every call, host side):
+ *   KS_FAULT_INJECT=alloc    every workspace allocation fails: the entry
+ *                            points that need one return KS_ERR_ALLOC before
+ *                            launching anything (ks_matmul reads the values in
+ *                            place instead);
+ *   KS_FAULT_INJECT=timeout  the tensor-core kernel's pipeline waits give up at
+ *                            once instead of after about one second: the kernel
+ *                            abandons its work (Y is unspecified), drains its
+ *                            copies, frees its tensor memory and returns, and
+ *                            the next ks_sync_status reports KS_ERR_TIMEOUT.
+ * Unset (or any other value), nothing is injected. */
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char *ks_last_error(void);

@@ -21,7 +21,7 @@ from ._lib import (KS_BF16, KS_F32, KS_TF32, KS_VARIANT_AUTO, KS_VARIANT_FMA,  #
 
 Pattern = Tuple[int, int, int, int]
 
-__all__ = ["matmul", "chain", "plan", "sync_status", "ks_dtype_of", "KsError", "VARIANTS"]
+__all__ = ["matmul", "chain", "plan", "sync_status", "workspace_info", "ks_dtype_of", "KsError", "VARIANTS"]
 
 
 def ks_dtype_of(t: torch.Tensor, tf32: bool = False) -> int:
@@ -222,6 +222,15 @@ def plan(pattern: Pattern, batch: int, dtype: int = KS_F32) -> str:
     a, b, c, d = (int(t) for t in pattern)
     _lib.check(_lib.load().ks_plan(a, b, c, d, int(batch), int(dtype), ctypes.byref(v)))
     return {v_: k for k, v_ in VARIANTS.items()}[v.value]
+
+
+def workspace_info() -> Tuple[int, int]:
+    """(allocations, reserved_bytes): workspace allocations the library has made
+    from its pools since the process started (all devices), and the device
+    memory the current device's pool holds now."""
+    n, r = ctypes.c_int64(0), ctypes.c_int64(0)
+    _lib.check(_lib.load().ks_workspace_info(ctypes.byref(n), ctypes.byref(r)))
+    return int(n.value), int(r.value)
 
 
 def sync_status(stream: Optional[torch.cuda.Stream] = None) -> None:

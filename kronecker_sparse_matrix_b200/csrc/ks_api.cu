@@ -9,7 +9,9 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "ks.h"
@@ -167,6 +169,29 @@ cudaMemPool_t chain_pool() {
     return pools[dev];
 }
 
+namespace {
+std::atomic<long long> g_pool_allocs{0};  // successful pool_alloc calls, all devices
+}  // namespace
+
+// KS_FAULT_INJECT=alloc: every workspace allocation fails (tests of the
+// KS_ERR_ALLOC paths).
+bool inject_alloc_failure() {
+    const char *f = getenv("KS_FAULT_INJECT");
+    return f && strcmp(f, "alloc") == 0;
+}
+
+cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t stream) {
+    if (inject_alloc_failure()) return cudaErrorMemoryAllocation;
+    cudaMemPool_t pool = chain_pool();
+    if (!pool) {
+        (void)cudaGetLastError();
+        return cudaErrorMemoryAllocation;
+    }
+    const cudaError_t e = cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
+    if (e == cudaSuccess) g_pool_allocs.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
 int sm_count() {
     static std::mutex mu;
     static int counts[64] = {};
@@ -187,6 +212,16 @@ ks_status record_error(ks_status s, const char *fmt, ...) {
     vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
     va_end(ap);
     return s;
+}
+
+ks_status matmul_no_workspace(const void *X, const void *V, int64_t a, int64_t b, int64_t c, int64_t d,
+                              int64_t batch, void *Y, int dtype, void *stream) {
+    Problem p;
+    bool noop = false;
+    ks_status s = make_problem(X, V, a, b, c, d, batch, Y, dtype, stream, &p, &noop);
+    if (s != KS_OK || noop) return s;
+    p.no_workspace = true;
+    return run(p, KS_VARIANT_AUTO);
 }
 
 }  // namespace ks
@@ -317,14 +352,9 @@ ks_status ks_chain_ep(const void *X, const void *const *factors, const ks_patter
     void *buf[2] = {nullptr, nullptr};
     const size_t bytes = ((size_t)batch * (size_t)widest * (size_t)elem + 255) / 256 * 256;
     const size_t total = n_factors > 2 ? 2 * bytes : bytes;
-    cudaMemPool_t pool = chain_pool();
-    if (!pool) {
-        (void)cudaGetLastError();
-        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
-    }
     {
         void *base = nullptr;
-        cudaError_t e = cudaMallocFromPoolAsync(&base, total, pool, st);
+        cudaError_t e = pool_alloc(&base, total, st);
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", total, cudaGetErrorString(e));
@@ -373,13 +403,8 @@ ks_status ks_matmul_dx(const void *dY, const void *values, int64_t a, int64_t b,
     if (ranges_overlap(dX, batch * in_f * elem, values, nvals * elem))
         return fail(KS_ERR_INVALID_ARG, "dX overlaps values");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaMemPool_t pool = chain_pool();
-    if (!pool) {
-        (void)cudaGetLastError();
-        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
-    }
     void *vt = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&vt, (size_t)(nvals * elem), pool, st);
+    cudaError_t e = pool_alloc(&vt, (size_t)(nvals * elem), st);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return fail(KS_ERR_ALLOC, "workspace allocation of %lld bytes failed: %s", (long long)(nvals * elem),
@@ -424,14 +449,9 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int6
     int splits = 1;
     long long rows_per_split = batch;
     dv_split(q, &splits, &rows_per_split);
-    cudaMemPool_t pool = chain_pool();
-    if (!pool) {
-        (void)cudaGetLastError();
-        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
-    }
     const size_t wbytes = (size_t)splits * (size_t)nvals * sizeof(float);
     void *w = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&w, wbytes, pool, st);
+    cudaError_t e = pool_alloc(&w, wbytes, st);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", wbytes, cudaGetErrorString(e));
@@ -453,8 +473,7 @@ ks_pattern butterfly_range(int p, int q, int L) {
 
 // Splits the range [p, q], whose product values are P, in the middle and fits
 // the two halves; recurses until single factors land in factors[k - 1].
-ks_status factorize_range(const float *P, int p, int q, int L, float *const *factors, cudaMemPool_t pool,
-                          cudaStream_t st) {
+ks_status factorize_range(const float *P, int p, int q, int L, float *const *factors, cudaStream_t st) {
     const int r = (p + q - 1) / 2;
     const ks_pattern p1 = butterfly_range(p, r, L), p2 = butterfly_range(r + 1, q, L);
     const int64_t n1 = p1.a * p1.b * p1.c * p1.d, n2 = p2.a * p2.b * p2.c * p2.d;
@@ -462,13 +481,13 @@ ks_status factorize_range(const float *P, int p, int q, int L, float *const *fac
     ks_status result = KS_OK;
     if (r == p) {
         v1 = factors[p - 1];
-    } else if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&v1), (size_t)n1 * 4, pool, st) != cudaSuccess) {
+    } else if (pool_alloc(reinterpret_cast<void **>(&v1), (size_t)n1 * 4, st) != cudaSuccess) {
         (void)cudaGetLastError();
         return fail(KS_ERR_ALLOC, "factorization workspace of %lld bytes", (long long)(n1 * 4));
     }
     if (r + 1 == q) {
         v2 = factors[q - 1];
-    } else if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&v2), (size_t)n2 * 4, pool, st) != cudaSuccess) {
+    } else if (pool_alloc(reinterpret_cast<void **>(&v2), (size_t)n2 * 4, st) != cudaSuccess) {
         (void)cudaGetLastError();
         result = fail(KS_ERR_ALLOC, "factorization workspace of %lld bytes", (long long)(n2 * 4));
     }
@@ -476,8 +495,8 @@ ks_status factorize_range(const float *P, int p, int q, int L, float *const *fac
         const cudaError_t e = launch_rank1_fit(P, v1, v2, p1.a, p1.b, p1.c, p2.b, p2.c, p2.d, st);
         if (e != cudaSuccess) result = cuda_fail(e, "rank-one fit launch");
     }
-    if (result == KS_OK && r > p) result = factorize_range(v1, p, r, L, factors, pool, st);
-    if (result == KS_OK && q > r + 1) result = factorize_range(v2, r + 1, q, L, factors, pool, st);
+    if (result == KS_OK && r > p) result = factorize_range(v1, p, r, L, factors, st);
+    if (result == KS_OK && q > r + 1) result = factorize_range(v2, r + 1, q, L, factors, st);
     if (r != p && v1) (void)cudaFreeAsync(v1, st);
     if (r + 1 != q && v2) (void)cudaFreeAsync(v2, st);
     return result;
@@ -504,14 +523,26 @@ ks_status ks_butterfly_factorize(const void *A, int log2n, void *const *factors,
         const cudaError_t e = cudaMemcpyAsync(factors[0], A, 4 * 4, cudaMemcpyDeviceToDevice, st);
         return e == cudaSuccess ? ok() : cuda_fail(e, "copy");
     }
-    cudaMemPool_t pool = chain_pool();
-    if (!pool) {
-        (void)cudaGetLastError();
-        return fail(KS_ERR_ALLOC, "workspace pool unavailable on this device");
-    }
     float *const *f = reinterpret_cast<float *const *>(factors);
-    const ks_status r = factorize_range(static_cast<const float *>(A), 1, log2n, log2n, f, pool, st);
+    const ks_status r = factorize_range(static_cast<const float *>(A), 1, log2n, log2n, f, st);
     return r == KS_OK ? ok() : r;
+}
+
+ks_status ks_workspace_info(int64_t *allocations, int64_t *reserved_bytes) {
+    if (allocations) *allocations = g_pool_allocs.load(std::memory_order_relaxed);
+    if (reserved_bytes) {
+        *reserved_bytes = 0;
+        cudaMemPool_t pool = chain_pool();
+        if (!pool) {
+            (void)cudaGetLastError();
+            return fail(KS_ERR_CUDA, "workspace pool unavailable on this device");
+        }
+        uint64_t v = 0;
+        const cudaError_t e = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &v);
+        if (e != cudaSuccess) return cuda_fail(e, "reading the pool's reserved memory");
+        *reserved_bytes = (int64_t)v;
+    }
+    return KS_OK;
 }
 
 const char *ks_last_error(void) { return g_msg; }

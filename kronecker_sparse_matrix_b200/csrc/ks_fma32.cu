@@ -522,17 +522,17 @@ cudaError_t launch_cfg_any(const Problem &p, const FmaConfig &c, const float *vt
 // workspace is freed on the stream after the kernel.  Measured against the
 // in-place path on the fp32 sweep: 1.20x median for d % 8 == 0; for smaller
 // l widths the gain (1.01-1.03x) did not cover the transpose on mid-size runs.
-// If the workspace cannot be had, the values are read in place.
+// If the workspace cannot be had, or the caller must not allocate
+// (Problem::no_workspace), the values are read in place.
 cudaError_t launch_fma32(const Problem &p, const FmaConfig &c_in) {
     // the l width comes from the caller's plan, the tile from this kernel's table
     const FmaConfig c = fma32_choose(p, c_in.dl);
     if (c.dl == 0) return cudaErrorInvalidConfiguration;
     const long long nvals = p.a * p.b * p.c * p.d;
     const double flops = 2.0 * (double)p.batch * (double)nvals;
-    if (c.dl == 8 && p.b % 4 == 0 && flops >= 1073741824.0 && nvals * 4 <= (64LL << 20)) {
-        cudaMemPool_t pool = chain_pool();
+    if (!p.no_workspace && c.dl == 8 && p.b % 4 == 0 && flops >= 1073741824.0 && nvals * 4 <= (64LL << 20)) {
         void *vt = nullptr;
-        if (pool && cudaMallocFromPoolAsync(&vt, (size_t)nvals * 4, pool, p.stream) == cudaSuccess) {
+        if (pool_alloc(&vt, (size_t)nvals * 4, p.stream) == cudaSuccess) {
             cudaError_t e = launch_transpose_blocks(p.V, vt, p.a * p.d, p.b, p.c, KS_F32, p.stream);
             if (e == cudaSuccess) e = launch_cfg_any(p, c, static_cast<const float *>(vt));
             const cudaError_t ef = cudaFreeAsync(vt, p.stream);

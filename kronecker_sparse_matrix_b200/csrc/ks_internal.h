@@ -21,6 +21,10 @@ struct Problem {
     // of the storage dtype (or is null), act is a ks_activation.
     const void *bias = nullptr;
     int act = 0;
+    // Set for callers that must not allocate: every kernel then works in the
+    // caller's buffers only (the fp32 kernel reads the values in place instead
+    // of staging a transposed copy in a pooled workspace).
+    bool no_workspace = false;
 
     int64_t in_features() const { return a * c * d; }
     int64_t out_features() const { return a * b * d; }
@@ -92,6 +96,14 @@ cudaError_t launch_rank1_fit(const float *P, float *V1, float *V2, int64_t a1, i
 
 // The library's retaining workspace pool of the current device (ks_api.cu).
 cudaMemPool_t chain_pool();
+// Stream-ordered allocation from chain_pool(); every successful one is counted
+// (ks_workspace_info).  Returns cudaErrorMemoryAllocation without a pool.
+cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t stream);
+
+// One validated KS product with Problem::no_workspace set (ks_api.cu; used by
+// ks_chain_noalloc).
+ks_status matmul_no_workspace(const void *X, const void *V, int64_t a, int64_t b, int64_t c, int64_t d,
+                              int64_t batch, void *Y, int dtype, void *stream);
 
 // Fused 4096-wide butterfly chain (ks_butterfly.cu): the twelve factors
 // (2^t, 2, 2, 2^(11-t)), t = 0..11, in that order.

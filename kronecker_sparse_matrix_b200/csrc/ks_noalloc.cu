@@ -75,9 +75,11 @@ extern "C" ks_status ks_chain_noalloc(const void *X, const void *const *factors,
     }
     if (batch == 0) return KS_OK;
     if (!X || !Y) return record_error(KS_ERR_INVALID_ARG, "X and Y must be non-null");
+    // Every product runs with Problem::no_workspace: the fp32 kernel reads the
+    // values in place instead of staging a transposed copy in a pooled workspace.
     if (n_factors == 1) {
         const ks_pattern &q = patterns[0];
-        return ks_matmul(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
+        return ks::matmul_no_workspace(X, factors[0], q.a, q.b, q.c, q.d, batch, Y, dtype, stream);
     }
     if (widest > (int64_t)(kHalfBytes / elem) / batch)
         return record_error(KS_ERR_INVALID_ARG,
@@ -93,7 +95,7 @@ extern "C" ks_status ks_chain_noalloc(const void *X, const void *const *factors,
     for (int t = 0; t < n_factors; ++t) {
         const ks_pattern &q = patterns[t];
         void *dst = (t == n_factors - 1) ? Y : static_cast<void *>(half[t & 1]);
-        ks_status s = ks_matmul(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, stream);
+        ks_status s = ks::matmul_no_workspace(src, factors[t], q.a, q.b, q.c, q.d, batch, dst, dtype, stream);
         if (s != KS_OK) return s;
         src = dst;
     }

@@ -1,7 +1,7 @@
 // sm_100a building blocks shared by the tensor-core kernels: mbarriers with
-// bounded waits, TMA tensor loads, tcgen05 tensor-memory allocation, MMA,
-// commit and loads, shared-memory matrix descriptors, and a 16-bit 8x8
-// register transpose.  Everything is inline PTX from the PTX ISA for sm_100a.
+// bounded waits, TMA tensor loads, tcgen05 tensor-memory allocation, MMA
+// (bf16 and TF32), commit and loads, shared-memory matrix descriptors, and a
+// 16-bit 8x8 register transpose.  Everything is inline PTX from the PTX ISA for sm_100a.
 #pragma once
 
 #include <cuda.h>
@@ -45,15 +45,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 // Waits for the phase of `parity` to complete.  Returns false if the CTA is
-// aborting or the wait ran out (which starts the abort).
+// aborting or the wait ran out after `bound_ns` (which starts the abort).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned *status) {
+                                          unsigned *status, uint64_t bound_ns = kTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (globaltimer() - t0 > bound_ns) {
             *abort_flag = 1;
             atomicOr(status, kDevTimeout);
             return false;
@@ -101,6 +101,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// TF32 inputs (fp32 words in shared memory, read by the tensor core at TF32
+// precision), fp32 accumulate: kind::tf32, K = 8 per instruction.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
@@ -124,6 +134,15 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
                  : "r"(taddr));
 #pragma unroll
     for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(r[q]);
+}
+// 4 consecutive fp32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = __uint_as_float(r[q]);
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 

@@ -125,6 +125,45 @@ def test_plan_is_host_only_and_sensible(lib):
     assert plan((3, 5, 7, 3), 10) == "stream"  # odd d: the scalar catch-all
 
 
+def test_plan_sends_tf32_and_bf16_to_the_tensor_cores(lib):
+    for p, n in [((1, 192, 48, 8), 25216), ((1, 256, 64, 16), 8192)]:
+        assert plan(p, n, _lib.KS_TF32) == "tc"
+        assert plan(p, n, _lib.KS_BF16) == "tc"
+        assert plan(p, n, _lib.KS_F32) == "fma"  # fp32 keeps fp32 arithmetic
+    for p in sweep_patterns():
+        assert plan(p, 25088, _lib.KS_TF32) == "tc"
+        assert plan(p, 25088, _lib.KS_BF16) == "tc"
+    # TF32's K step is 8 j, bf16's 16
+    assert plan((1, 64, 8, 1), 1000, _lib.KS_TF32) == "tc"
+    assert plan((1, 64, 8, 1), 1000, _lib.KS_BF16) == "fma"
+    assert plan((1, 64, 12, 1), 1000, _lib.KS_TF32) == "fma"
+    assert plan((1, 64, 64, 3), 1000, _lib.KS_TF32) != "tc"  # d = 3: no l width for the tensor-core tiles
+    for p in butterfly_patterns(12):
+        assert plan(p, 4096, _lib.KS_TF32) == "stream"
+
+
+def test_tc_variant_refuses_fp32(lib):
+    v = ctypes.c_int(-1)
+    assert lib.ks_plan(1, 64, 64, 1, 100, _lib.KS_F32, ctypes.byref(v)) == 0 and v.value == _lib.KS_VARIANT_FMA
+    # forcing the tensor cores on KS_F32 is refused before any device call
+    assert lib.ks_matmul_variant(P, P * 2, 1, 64, 64, 1, 100, P * 4, _lib.KS_F32, _lib.KS_VARIANT_TC, None) == 3
+    assert b"KS_TF32" in lib.ks_last_error()
+
+
+def test_injected_allocation_failure_is_reported_before_any_launch(lib, monkeypatch):
+    monkeypatch.setenv("KS_FAULT_INJECT", "alloc")
+    pats = (_lib.KsPattern * 2)(_lib.KsPattern(1, 4, 4, 2), _lib.KsPattern(2, 4, 4, 1))
+    ptrs = (ctypes.c_void_p * 2)(P * 2, P * 3)
+    assert lib.ks_chain(P, ptrs, pats, 2, 4, P * 4, 0, None) == 4
+    assert b"workspace" in lib.ks_last_error()
+    assert lib.ks_matmul_dx(P, P * 2, 2, 2, 2, 2, 4, P * 4, 0, None) == 4
+    assert lib.ks_matmul_dv(P, P * 2, 2, 2, 2, 2, 4, P * 4, 0, None) == 4
+    facs = (ctypes.c_void_p * 4)(P * 4, P * 5, P * 6, P * 7)
+    assert lib.ks_butterfly_factorize(P, 4, facs, 0, None) == 4
+    n = ctypes.c_int64(-1)
+    assert lib.ks_workspace_info(ctypes.byref(n), None) == 0 and n.value == 0  # nothing was ever allocated
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(_lib, "_lib", None)

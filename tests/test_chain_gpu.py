@@ -35,17 +35,33 @@ def test_small_chains(patterns, dtype):
     Y = ks.chain(c.X.to(DEV), [f.to(DEV) for f in c.factors], patterns)
     ks.sync_status()
     ref = oracle.chain(c.X, c.factors, patterns)
-    tol = 1e-5 if dtype == torch.float32 else 3e-2  # bf16: one rounding per factor
+    # bf16: every intermediate is rounded to bf16 too; measured on B200 at most
+    # 5.7e-3 on these chains (4 seeds, 45 and 1000 rows), inside the 1e-2 bound
+    tol = 1e-5 if dtype == torch.float32 else 1e-2
     assert oracle.max_rel_err(Y.cpu(), ref) <= tol
 
 
-def test_butterfly_chain_full_size_sampled_rows():
-    c = inputs.butterfly(device=DEV)
+def test_unfused_bf16_butterfly_within_its_rounding_bound():
+    """Factor by factor, a bf16 chain of n factors rounds n - 1 intermediates
+    to bf16 (relative error at most 2^-9 each, round to nearest even) before
+    the output's own rounding: the bound is n * 2^-9, 2.3e-2 for the twelve
+    factors of the 4096-wide butterfly (measured 1.1e-2).  The fused kernel,
+    the default for this chain, keeps fp32 intermediates and meets 1e-2."""
+    c = inputs.butterfly(device=DEV, dtype=torch.bfloat16, batch=512, seed=3)
+    Y = ks.chain(c.X, c.factors, c.patterns, fused=False)
+    ks.sync_status()
+    ref = oracle.chain(c.X.cpu(), [f.cpu() for f in c.factors], c.patterns)
+    assert oracle.max_rel_err(Y.cpu(), ref) <= len(c.patterns) * 2.0 ** -9
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_butterfly_chain_full_size_every_row(dtype):
+    c = inputs.butterfly(device=DEV, dtype=dtype)
     Y = ks.chain(c.X, c.factors, c.patterns)
     ks.sync_status()
-    rows = [0, 1, 17, 1000, 2048, 4095]
-    ref = oracle.chain(c.X[rows].cpu(), [f.cpu() for f in c.factors], c.patterns)
-    assert oracle.max_rel_err(Y[rows].cpu(), ref) <= 1e-5
+    ref = oracle.chain(c.X.cpu(), [f.cpu() for f in c.factors], c.patterns)
+    tol = 1e-5 if dtype == torch.float32 else 1e-2  # fused: fp32 intermediates, one output rounding
+    assert oracle.max_rel_err(Y.cpu(), ref) <= tol
 
 
 def test_chain_of_one_equals_matmul():

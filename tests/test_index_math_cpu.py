@@ -111,43 +111,204 @@ def test_fma32_copies_cover_a_stage_once(tile):
 
 
 # ------------------------------------------------------------------ ks_tc.cu
-def chunk_j(dls):
-    return 16 if dls == 8 else 64 // dls
+# es = element bytes: 2 (bf16, kind::f16) or 4 (fp32 read as TF32, kind::tf32).
+def chunk_j(dls, es=2):
+    return (32 if dls == 8 else 128 // dls) // es
+
+
+def group_stride(es):
+    return 144 if es == 2 else 256
+
+
+def octet_stride(es):
+    return 16 * 144 if es == 2 else 128 * 32
+
+
+def plane_stride(dls, es):
+    return (chunk_j(dls, es) // 8) * octet_stride(es)
+
+
+def slot_bytes(dls, es):
+    raw = 128 * chunk_j(dls, es) * dls * es
+    return (raw if dls == 1 else dls * plane_stride(dls, es) + 1023) // 1024 * 1024
 
 
 def tc_task_unit(dls, task, units):
+    """bf16 transposer: task -> (raw unit q, group g of 8 rows)."""
     if dls == 8:
         return task % units, task // units
     q = task & 7
     return q, ((task >> 3) + (q >> (1 if dls == 2 else 2))) & 15
 
 
+def bf16_transposer_writes(dls):
+    """(q, g, e) -> plane address of output unit e of a bf16 task."""
+    es, ctj = 2, chunk_j(dls, 2)
+    out = {}
+    for q in range(ctj * dls * es // 16):
+        for g in range(16):
+            for e in range(8):
+                f = 8 * q + e
+                j, l = f // dls, f % dls
+                out[(q, g, e)] = l * plane_stride(dls, es) + (j >> 3) * octet_stride(es) + g * group_stride(es) + \
+                    (j & 7) * 16
+    return out
+
+
 @pytest.mark.parametrize("dls", [2, 4, 8])
-def test_tc_transposer_quarter_warps_reach_eight_bank_groups(dls):
-    ctj = chunk_j(dls)
-    units = ctj * dls // 8
+def test_tc_bf16_transposer_quarter_warps_reach_eight_bank_groups(dls):
+    es, ctj = 2, chunk_j(dls, 2)
+    units = ctj * dls * es // 16
     tasks = 16 * units // 128
-    group_stride, octet_stride = 144, 16 * 144
-    slot = dls * (ctj // 8) * octet_stride
+    slot = slot_bytes(dls, es)
+    assert slot >= 128 * ctj * dls * es  # the in-place planes cover the raw chunk
+    wr = bf16_transposer_writes(dls)
     written, mapped = set(), set()
     for k in range(tasks):
         for t0 in range(0, 128, 8):  # one quarter-warp: 8 consecutive lanes
             qg = [tc_task_unit(dls, t + 128 * k, units) for t in range(t0, t0 + 8)]
             for r in range(8):  # reads of the raw chunk
-                groups = {((g8 * 8 + r) * units + q) % 8 for q, g8 in qg}
+                groups = {((g * 8 + r) * units + q) % 8 for q, g in qg}
                 assert len(groups) == 8
             for e in range(8):  # writes of the padded planes
                 addrs = []
-                for q, g8 in qg:
-                    f = 8 * q + e
-                    j, l = f // dls, f % dls
-                    a = (l * (ctj // 8) + (j >> 3)) * octet_stride + g8 * group_stride + (j & 7) * 16
+                for q, g in qg:
+                    a = wr[(q, g, e)]
                     assert 0 <= a and a + 16 <= slot and a not in written
                     written.add(a)
                     addrs.append(a)
                 assert len({(a // 16) % 8 for a in addrs}) == 8
             mapped.update(qg)
     assert len(mapped) == tasks * 128 and all(0 <= q < units and 0 <= g < 16 for q, g in mapped)
+
+
+@pytest.mark.parametrize("dls", [2, 4, 8])
+def test_tc_bf16_mma_descriptor_reads_what_the_transposer_wrote(dls):
+    """bf16 A operand of one MMA (plane l, K step s): the canonical MN-major
+    no-swizzle layout, element (row m, k) at start + (m // 8) * SBO +
+    (k // 8) * LBO + (k % 8) * 16 + (m % 8) * 2, start = l * PS + 2 s OS,
+    LBO = OS, SBO = GS; it must land on X[row m][j = 16 s + k][l]."""
+    es, ctj = 2, chunk_j(dls, 2)
+    wr = bf16_transposer_writes(dls)
+    where = {}
+    for (q, g, e), a in wr.items():
+        f = 8 * q + e
+        j, l = f // dls, f % dls
+        for r in range(8):
+            where[(g * 8 + r, j, l)] = a + r * es
+    assert len(where) == 128 * ctj * dls and len(set(where.values())) == len(where)
+    os_, gs, ps = octet_stride(es), group_stride(es), plane_stride(dls, es)
+    for l in range(dls):
+        for s in range(ctj // 16):
+            start = l * ps + 2 * s * os_
+            for m in range(128):
+                for k in range(16):
+                    addr = start + (m // 8) * gs + (k // 8) * os_ + (k % 8) * 16 + (m % 8) * es
+                    assert addr == where[(m, 16 * s + k, l)]
+
+
+def tf32_tasks(dls):
+    """The fp32 transposer of ks_tc.cu, modelled per thread t (0..127) and task
+    k: the raw addresses it reads (one list per load instruction) and, per
+    output unit, the plane address and the (row, j, l) of its four words."""
+    ctj = chunk_j(dls, 4)
+    jqn, lqn = ctj // 4, (2 if dls == 8 else 1)
+    tpr = jqn * lqn
+    rb = ctj * dls * 4
+    ps, os_ = plane_stride(dls, 4), octet_stride(4)
+    out = {}
+    for t in range(128):
+        for k in range(tpr):
+            task = t + 128 * k
+            lq, jq, n = task % lqn, (task // lqn) % jqn, task // tpr
+            reads, units = [], []
+            if dls == 2:
+                sw = n & 1
+                reads = [n * rb + (2 * jq + sw) * 16, n * rb + (2 * jq + 1 - sw) * 16]
+                words = {0: [(n, 4 * jq + w, 0) for w in range(4)], 1: [(n, 4 * jq + w, 1) for w in range(4)]}
+                les = [0, 1]
+            else:
+                rot = ((jq + 2 * (n & 1)) & 3) if dls == 8 else (n & 3)
+                for i in range(4):
+                    j = 4 * jq + ((i + rot) & 3)
+                    reads.append(n * rb + (j * (dls // 4) + lq) * 16)
+                words = {e: [(n, 4 * jq + w, 4 * lq + e) for w in range(4)] for e in range(4)}
+                les = [0, 1, 2, 3]
+            half = (jq & 1) ^ ((n >> 2) & 1)
+            for e in les:
+                addr = (jq >> 1) * os_ + n * 32 + half * 16 + (4 * lq + e) * ps
+                units.append((addr, words[e]))
+            out[(t, k)] = (reads, units)
+    return out, tpr
+
+
+@pytest.mark.parametrize("dls", [2, 4, 8])
+def test_tc_tf32_transposer_covers_the_planes_and_spreads_bank_groups(dls):
+    """Every element of the raw chunk lands once in the planes, which fit the
+    slot; each quarter-warp's reads reach eight bank groups, its writes at
+    least four (a 16-byte store of eight lanes in at most two wavefronts)."""
+    ctj = chunk_j(dls, 4)
+    tasks, tpr = tf32_tasks(dls)
+    slot = slot_bytes(dls, 4)
+    placed = {}
+    for (t, k), (reads, units) in tasks.items():
+        for addr, words in units:
+            assert 0 <= addr and addr + 16 <= slot
+            for w, elem in enumerate(words):
+                assert elem not in placed
+                placed[elem] = addr + 4 * w
+    assert len(placed) == 128 * ctj * dls and len(set(placed.values())) == len(placed)
+    for k in range(tpr):
+        for t0 in range(0, 128, 8):
+            lanes = [tasks[(t, k)] for t in range(t0, t0 + 8)]
+            for i in range(len(lanes[0][0])):
+                assert len({(r[0][i] // 16) % 8 for r in lanes}) == 8
+            for u in range(len(lanes[0][1])):
+                groups = [(r[1][u][0] // 16) % 8 for r in lanes]
+                assert max(groups.count(g) for g in groups) <= 2
+
+
+def test_tc_tf32_raw_reads_pick_the_right_elements():
+    """The raw chunk holds row n's (j, l) at n * rb + (j * dls + l) * 4; the
+    words the model assigns to each output unit are the ones the reads fetch."""
+    for dls in (2, 4, 8):
+        ctj = chunk_j(dls, 4)
+        rb = ctj * dls * 4
+        tasks, _ = tf32_tasks(dls)
+        for (t, k), (reads, units) in tasks.items():
+            fetched = set()
+            for r in reads:
+                n, off = divmod(r, rb)
+                for w in range(4):
+                    f = off // 4 + w
+                    fetched.add((n, f // dls, f % dls))
+            assert fetched == {elem for _, words in units for elem in words}
+
+
+@pytest.mark.parametrize("dls", [2, 4, 8])
+def test_tc_tf32_mma_descriptor_reads_what_the_transposer_wrote(dls):
+    """TF32 A operand of one MMA (plane l, K step s): the canonical K-major
+    layout with the 32-byte swizzle, element (row m, k) at start + (m // 8) *
+    SBO + (m % 8) * 32 + k * 4 with address bit 4 flipped by bit 7 (within
+    the 256-byte atom), start = l * PS + s * OS (256-byte aligned), SBO = 256.
+    It must land on X[row m][j = 8 s + k][l]."""
+    ctj = chunk_j(dls, 4)
+    tasks, _ = tf32_tasks(dls)
+    placed = {}
+    for reads, units in tasks.values():
+        for addr, words in units:
+            for w, elem in enumerate(words):
+                placed[elem] = addr + 4 * w
+    ps, os_ = plane_stride(dls, 4), octet_stride(4)
+    for l in range(dls):
+        for s in range(ctj // 8):
+            start = l * ps + s * os_
+            assert start % 256 == 0
+            for m in range(128):
+                for k in range(8):
+                    addr = start + (m // 8) * 256 + (m % 8) * 32 + k * 4
+                    addr ^= ((addr >> 7) & 1) << 4
+                    assert addr == placed[(m, 8 * s + k, l)]
 
 
 def tc_bp(dls, b):
@@ -157,28 +318,35 @@ def tc_bp(dls, b):
     return 0
 
 
-def tc_kc(dls, bp):
-    for kc in range(min(bp, 64 // dls), 7, -8):
-        if bp % kc == 0 and dls * kc == 64:
+def tc_kc(dls, bp, es=2):
+    ce = 128 // es
+    kcm = ce // dls
+    lw = min(8, kcm)
+    for kc in range(min(bp, kcm) // lw * lw, lw - 1, -lw):
+        if bp % kc == 0 and dls * kc == ce:
             return kc
-    for kc in range(min(bp, 64 // dls), 7, -8):
+    for kc in range(min(bp, kcm) // lw * lw, lw - 1, -lw):
         if bp % kc == 0:
             return kc
     return 0
 
 
+@pytest.mark.parametrize("es", [2, 4])
 @pytest.mark.parametrize("p", [(2, 48, 48, 2), (1, 48, 48, 4), (2, 64, 64, 16), (1, 192, 48, 8), (3, 32, 16, 4),
-                               (1, 256, 256, 2), (2, 48, 48, 1), (1, 16, 16, 1), (1, 96, 96, 4), (1, 80, 16, 2)])
-def test_tc_epilogue_writes_each_output_once(p):
+                               (1, 256, 256, 2), (2, 48, 48, 1), (1, 16, 16, 1), (1, 96, 96, 4), (1, 80, 16, 2),
+                               (1, 48, 8, 1), (2, 256, 64, 16)])
+def test_tc_epilogue_writes_each_output_once(p, es):
     """The output boxes of a tile: 32 rows x (DLS * kc) elements per warp and
     chunk, either one tensor store of a contiguous box (d == DLS) or 16-byte
     stores of its units; N = 300 leaves a ragged last row block."""
     a, b, c, d = p
     dls = 8 if d % 8 == 0 else d
     bp = tc_bp(dls, b)
-    kc = tc_kc(dls, bp)
+    kc = tc_kc(dls, bp, es)
+    assert kc > 0 and bp % kc == 0 and dls * kc * es <= 128
+    rpu = 16 // es
     n, out_f = 300, a * b * d
-    units = dls * kc // 8
+    units = dls * kc * es // 16
     written = collections.Counter()
     for i in range(a):
         for gl in range(d // dls):
@@ -194,7 +362,7 @@ def test_tc_epilogue_writes_each_output_once(p):
                                 if row0 >= n:
                                     continue
                                 x = ybase + kq * d
-                                assert (x * 2) % 16 == 0
+                                assert (x * es) % 16 == 0
                                 for r in range(min(32, n - row0)):
                                     for e in range(dls * kc):
                                         written[(row0 + r, x + e)] += 1
@@ -203,9 +371,33 @@ def test_tc_epilogue_writes_each_output_once(p):
                                     u = lane & 7
                                     if u >= units:
                                         continue
-                                    col = ybase + (kq + 8 * u // dls) * d + (8 * u) % dls
+                                    col = ybase + (kq + rpu * u // dls) * d + (rpu * u) % dls
                                     for r in range(lane >> 3, min(32, n - row0), 4):
-                                        for e in range(8):
+                                        for e in range(rpu):
                                             written[(row0 + r, col + e)] += 1
     assert all(0 <= r < n and 0 <= col < out_f for r, col in written)
     assert len(written) == n * out_f and set(written.values()) == {1}
+
+
+@pytest.mark.parametrize("es", [2, 4])
+@pytest.mark.parametrize("dls", [1, 2, 4, 8])
+def test_tc_shared_memory_offsets_keep_their_alignment(dls, es):
+    """Every X ring slot is a TMA destination (128-byte aligned at least, 1 KiB
+    for the 128-byte swizzle of d = 1), and the values ring that follows the X
+    ring holds swizzle atoms of 8 rows x the row width, which must sit at
+    multiples of their size: slot sizes and values planes keep 1 KiB / atom
+    alignment for every ring depth and pass width."""
+    ctj = chunk_j(dls, es)
+    slot = slot_bytes(dls, es)
+    assert slot % 1024 == 0
+    row = ctj * es  # values row bytes: the swizzle width
+    assert row in (32, 64, 128)
+    atom = 8 * row
+    for bp in range(16, min(256, 512 // dls) + 1, 16):
+        plane = bp * ctj * es
+        vstage = plane * dls
+        for stages in range(2, 9):
+            off_v = stages * slot
+            for vs in range(4):
+                for l in range(dls):
+                    assert (off_v + vs * vstage + l * plane) % atom == 0

@@ -94,7 +94,8 @@ def test_stream_kernel_bf16(p):
 
 
 @pytest.mark.parametrize("p", [(1, 192, 48, 8), (2, 64, 64, 2)])
-def test_tf32_dtype_meets_its_tolerance(p):
+def test_tf32_dtype_runs_on_the_tensor_cores(p):
+    assert ks.plan(p, 100, ks.KS_TF32) == "tc"
     run_and_check(p, 100, tf32=True)
 
 
@@ -158,13 +159,12 @@ def sampled_rows(batch, k=48, seed=1):
 
 
 @pytest.mark.parametrize("name,dtype", [("vit", torch.float32), ("gpt2", torch.float32), ("gpt2", torch.bfloat16)])
-def test_full_size_configs_sampled_rows(name, dtype):
+def test_full_size_configs_every_row(name, dtype):
     f = getattr(inputs, name)(dtype=dtype, device=DEV)
     Y = ks.matmul(f.X, f.values, f.pattern)
     ks.sync_status()
-    rows = sampled_rows(f.batch)
-    ref = oracle.matmul(f.X[rows].cpu(), f.values.cpu(), f.pattern)
-    assert oracle.max_rel_err(Y[rows].cpu(), ref) <= TOL[dtype]
+    ref = oracle.matmul(f.X.cpu(), f.values.cpu(), f.pattern)
+    assert oracle.max_rel_err(Y.cpu(), ref) <= TOL[dtype]
 
 
 @pytest.mark.parametrize("idx", [0, 38, 77, 120, 150, 200, 229, 257])
@@ -176,6 +176,25 @@ def test_full_size_sweep_patterns_sampled_rows(idx, dtype):
     rows = sampled_rows(f.batch, k=24)
     ref = oracle.matmul(f.X[rows].cpu(), f.values.cpu(), p)
     assert oracle.max_rel_err(Y[rows].cpu(), ref) <= TOL[dtype]
+
+
+# Full-size sweep patterns compared on every row: the tensor-core kernel's l
+# widths 1 (48 and 256 x 64 blocks, a = 64 and 8), 2, 4, 8 with d = 8 (whole
+# 256-byte rows) and 8 with d >= 16 (four-dimensional boxes), the last with
+# several k passes per X tile (b = 96, 128 with d = 16, 32); the fp32 kernel's
+# l widths 1, 2, 4, 8 (d >= 16 with the transposed-values workspace).
+FULL_ROWS = [82, 205, 127, 48, 248, 117, 36, 234]
+
+
+@pytest.mark.parametrize("idx", FULL_ROWS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_full_size_sweep_patterns_every_row(idx, dtype):
+    p = inputs.sweep_patterns()[idx]
+    f = inputs.sweep_inputs(idx, dtype=dtype, device=DEV)
+    Y = ks.matmul(f.X, f.values, p)
+    ks.sync_status()
+    ref = oracle.matmul(f.X.cpu(), f.values.cpu(), p)
+    assert oracle.max_rel_err(Y.cpu(), ref) <= TOL[dtype], p
 
 
 TC_CASES = [(1, 64, 64, 1), (1, 48, 48, 1), (2, 64, 64, 2), (1, 256, 64, 16), (1, 96, 96, 4), (4, 128, 128, 1),

@@ -61,3 +61,27 @@ def test_noalloc_largest_fitting_chain_then_rejects_one_row_more():
     with pytest.raises(ks.KsError) as err:
         chain_noalloc(x, c.factors, pats)
     assert err.value.status == 1 and "scratch" in str(err.value)
+
+
+def test_noalloc_takes_no_workspace_where_ks_matmul_would():
+    """Factor (1, 256, 256, 64) at batch 256 is an fp32 product that ks_matmul
+    runs with a pooled workspace (a transposed copy of its 16 MiB of values);
+    its 16 MiB intermediate fits the fixed scratch exactly.  Through
+    ks_chain_noalloc the library's workspace count must not move, and the
+    result must still match ks_chain's."""
+    pats = [(1, 256, 256, 64), (64, 16, 16, 16)]
+    c = inputs.chain_inputs(pats, 256, seed=5, device=DEV)
+    n0, _ = ks.workspace_info()
+    ks.matmul(c.X, c.factors[0], pats[0])
+    ks.sync_status()
+    n1, _ = ks.workspace_info()
+    assert n1 == n0 + 1  # ks_matmul took its workspace for this factor
+    for _ in range(2):
+        y = chain_noalloc(c.X, c.factors, pats)
+        ks.sync_status()
+        assert ks.workspace_info()[0] == n1
+    y_ref = ks.chain(c.X, c.factors, pats)
+    assert oracle.max_rel_err(y, y_ref.double()) <= 1e-5
+    rows = [0, 1, 100, 255]
+    ref = oracle.chain(c.X[rows].cpu(), [f.cpu() for f in c.factors], pats)
+    assert oracle.max_rel_err(y[rows].cpu(), ref) <= 1e-5
