@@ -162,6 +162,15 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b,
                        int64_t c, int64_t d, int64_t batch, void *dV, int dtype,
                        void *stream);
 
+/* Bias gradient of the page's KSLinear layer, y = x K^T + bias:
+ *     db[col] = sum_{n<batch} dY[n][col],  col < width.
+ * dY is batch x width (DEVICE, row-major), db width elements (DEVICE), one
+ * dtype; db must not overlap dY.  Sums are fp32, over row ranges in row order,
+ * the ranges' partial sums (a stream-ordered fp32 workspace from the
+ * library's pool, KS_ERR_ALLOC if it cannot be had) added in range order: the
+ * result is deterministic; bf16 db is rounded once.  batch == 0 writes zeros. */
+ks_status ks_bias_grad(const void *dY, int64_t batch, int64_t width, void *db, int dtype, void *stream);
+
 /* What KS_VARIANT_AUTO would run for this problem, written to *variant
  * (a ks_variant).  Host-only: touches no device. */
 ks_status ks_plan(int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
@@ -270,8 +279,8 @@ ks_status ks_workspace_info(int64_t *allocations, int64_t *reserved_bytes);
  * thread issues iters x 8 packed FMAs (fma.rn.f32x2, four flops each), so a
  * launch is blocks * 256 * iters * 32 flop.  out is a DEVICE array of
  * `blocks` floats (a checksum per block, so no work is optimised away).
- * Time it with events on `stream`.  KS_ERR_INVALID_ARG for a null out or
- * non-positive blocks / iters. */
+ * Time it with events on `stream`.  KS_ERR_INVALID_ARG for a null out,
+ * non-positive blocks, or iters not a positive multiple of 16. */
 ks_status ks_fma_rate_probe(float *out, int blocks, int64_t iters, void *stream);
 
 /* Fault injection for tests (read on every call, host side):

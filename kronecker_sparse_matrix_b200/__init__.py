@@ -127,6 +127,23 @@ def matmul_dv(dy: torch.Tensor, x: torch.Tensor, pattern: Pattern, *, out: Optio
     return out
 
 
+def bias_grad(dy: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Column sums of dY (batch, width): the bias gradient of y = x K^T + bias
+    (fp32 sums in a fixed order; bf16 rounded once)."""
+    if dy.dim() != 2 or not dy.is_cuda or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous 2-D CUDA tensor")
+    if out is None:
+        out = torch.empty(dy.shape[1], dtype=dy.dtype, device=dy.device)
+    elif out.numel() != dy.shape[1] or out.dtype != dy.dtype or out.device != dy.device or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor of width elements with dy's dtype and device")
+    with torch.cuda.device(dy.device):
+        st = _lib.load().ks_bias_grad(dy.data_ptr(), dy.shape[0], dy.shape[1], out.data_ptr(), ks_dtype_of(dy),
+                                      _stream_ptr(stream, dy.device))
+    _lib.check(st)
+    return out
+
+
 def butterfly_factorize(a: torch.Tensor, *, stream: Optional[torch.cuda.Stream] = None):
     """Fit a dense 2^L x 2^L fp32 CUDA matrix A (the K of Y = X K^T) with the L
     butterfly factors; returns (factors, patterns) for chain(), factor 0 first."""
@@ -160,14 +177,14 @@ class _KSLinearFn(torch.autograd.Function):
         dy = dy.contiguous()
         dx = matmul_dx(dy, values.contiguous(), ctx.pattern) if ctx.needs_input_grad[0] else None
         dv = matmul_dv(dy, x, ctx.pattern).view(values.shape) if ctx.needs_input_grad[1] else None
-        db = dy.sum(0) if ctx.needs_input_grad[2] else None
+        db = bias_grad(dy) if ctx.needs_input_grad[2] else None
         return dx, dv, db, None
 
 
 class KSLinear(torch.nn.Module):
     """A linear layer whose weight is one KS factor of pattern (a, b, c, d):
     in_features a*c*d, out_features a*b*d, y = x K^T (+ bias, fused into the
-    product's epilogue; its gradient is the column sum of dY).  The values are
+    product's epilogue; its gradient is the column sum of dY, ks_bias_grad).  The values are
     a parameter of shape (a, d, b, c), drawn N(0, 1/c) (unit-variance outputs
     for unit-variance inputs).  Leading dimensions of x are flattened."""
 

@@ -47,6 +47,7 @@ SIGNATURES = {
     "ks_matmul_dv": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_chain_ex": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _int, _vp]),
     "ks_chain_noalloc": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
+    "ks_bias_grad": (_int, [_vp, _i64, _i64, _vp, _int, _vp]),
     "ks_workspace_info": (_int, [ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "ks_fma_rate_probe": (_int, [_vp, _int, _i64, _vp]),
     "ks_last_error": (ctypes.c_char_p, []),

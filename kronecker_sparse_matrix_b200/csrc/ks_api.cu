@@ -464,6 +464,42 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int6
     return result == KS_OK ? ok() : result;
 }
 
+ks_status ks_bias_grad(const void *dY, int64_t batch, int64_t width, void *db, int dtype, void *stream) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    if (batch < 0 || width <= 0) return fail(KS_ERR_INVALID_ARG, "need batch >= 0 and width > 0");
+    int64_t cells = 0;
+    if (!mul_ok(std::max<int64_t>(batch, 1), width, &cells) || !mul_ok(cells, 4, &cells))
+        return fail(KS_ERR_INVALID_ARG, "sizes overflow int64");
+    if (!db) return fail(KS_ERR_INVALID_ARG, "db must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    if ((s = check_align(db, elem, "db")) != KS_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (batch == 0) {  // an empty sum
+        cudaError_t e = cudaMemsetAsync(db, 0, (size_t)(width * elem), st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "db clear");
+    }
+    if (!dY) return fail(KS_ERR_INVALID_ARG, "dY must be non-null");
+    if ((s = check_align(dY, elem, "dY")) != KS_OK) return s;
+    if (ranges_overlap(db, width * elem, dY, batch * width * elem)) return fail(KS_ERR_INVALID_ARG, "db overlaps dY");
+    int splits = 1;
+    long long rows_per_split = batch;
+    colsum_split(batch, width, &splits, &rows_per_split);
+    const size_t wbytes = (size_t)splits * (size_t)width * sizeof(float);
+    void *w = nullptr;
+    cudaError_t e = pool_alloc(&w, wbytes, st);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", wbytes, cudaGetErrorString(e));
+    }
+    ks_status result = KS_OK;
+    e = launch_colsum(dY, db, batch, width, dtype, static_cast<float *>(w), splits, rows_per_split, st);
+    if (e != cudaSuccess) result = cuda_fail(e, "column-sum launch");
+    e = cudaFreeAsync(w, st);
+    if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+    return result;
+}
+
 namespace {
 
 // The product of butterfly factors F_p .. F_q of size 2^L (F_k = (2^(k-1), 2, 2, 2^(L-k))).

@@ -11,6 +11,9 @@
 //                for each (i, l) a (b x N) x (N x c) product, reduced over the
 //                batch: dv_kernel below, split over row ranges, then a
 //                reduction of the fp32 partial sums in a fixed order.
+//   dbias:       db[col] = sum_n dY[n, col], the gradient of the layer's bias:
+//                column sums over row ranges (colsum_kernel), reduced in the
+//                same fixed order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -267,7 +270,67 @@ cudaError_t launch_dv_dl(const DvProblem &q, float *W, int splits, long long row
     }
 }
 
+// Column sums of dY over one row range: thread = column (consecutive threads
+// read consecutive columns of a row), blockIdx.y = range; fp32 sums in row
+// order into W[range][col].
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_kernel(const T *__restrict__ dY, float *__restrict__ W, long long N,
+                                                     long long width, long long rows_per_split) {
+    const long long col = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (col >= width) return;
+    const long long r0 = (long long)blockIdx.y * rows_per_split;
+    const long long r1 = min(N, r0 + rows_per_split);
+    const T *p = dY + r0 * width + col;
+    float s = 0.f;
+    long long r = r0;
+    for (; r + 4 <= r1; r += 4, p += 4 * width) {  // four independent loads in flight
+        const float v0 = ld_f(p), v1 = ld_f(p + width), v2 = ld_f(p + 2 * width), v3 = ld_f(p + 3 * width);
+        s += v0;
+        s += v1;
+        s += v2;
+        s += v3;
+    }
+    for (; r < r1; ++r, p += width) s += ld_f(p);
+    W[(long long)blockIdx.y * width + col] = s;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_reduce_kernel(const float *__restrict__ W, T *__restrict__ db,
+                                                            long long width, int splits) {
+    const long long col = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (col >= width) return;
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += W[(long long)k * width + col];
+    st_f(db + col, s);
+}
+
 }  // namespace
+
+void colsum_split(long long batch, long long width, int *splits, long long *rows_per_split) {
+    const long long col_blocks = (width + 255) / 256;
+    long long want = std::max<long long>(1, (4LL * sm_count() + col_blocks - 1) / col_blocks);
+    want = std::min<long long>(want, std::max<long long>(1, batch / 64));  // at least 64 rows per range
+    want = std::min<long long>(want, 65535);
+    const long long rows = (batch + want - 1) / want;
+    *rows_per_split = rows;
+    *splits = (int)((batch + rows - 1) / rows);
+}
+
+cudaError_t launch_colsum(const void *dY, void *db, long long batch, long long width, int dtype, float *W, int splits,
+                          long long rows_per_split, cudaStream_t stream) {
+    const dim3 grid((unsigned)((width + 255) / 256), (unsigned)splits);
+    const unsigned rgrid = (unsigned)((width + 255) / 256);
+    if (dtype == KS_BF16) {
+        colsum_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(dY), W, batch,
+                                                                width, rows_per_split);
+        colsum_reduce_kernel<__nv_bfloat16><<<rgrid, 256, 0, stream>>>(W, static_cast<__nv_bfloat16 *>(db), width,
+                                                                      splits);
+    } else {
+        colsum_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float *>(dY), W, batch, width, rows_per_split);
+        colsum_reduce_kernel<float><<<rgrid, 256, 0, stream>>>(W, static_cast<float *>(db), width, splits);
+    }
+    return cudaGetLastError();
+}
 
 int dv_dl(int64_t d) { return d % 8 == 0 ? 8 : d % 4 == 0 ? 4 : d % 2 == 0 ? 2 : 1; }
 

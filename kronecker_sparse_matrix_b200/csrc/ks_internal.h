@@ -83,6 +83,11 @@ struct DvProblem {
 int dv_dl(int64_t d);
 void dv_split(const DvProblem &q, int *splits, long long *rows_per_split);
 cudaError_t launch_dv(const DvProblem &q, float *W, int splits, long long rows_per_split);
+// Column sums db[col] = sum_n dY[n][col] (ks_backward.cu): fp32 partial sums
+// over `splits` row ranges into W[split][width], then added in range order.
+void colsum_split(long long batch, long long width, int *splits, long long *rows_per_split);
+cudaError_t launch_colsum(const void *dY, void *db, long long batch, long long width, int dtype, float *W, int splits,
+                          long long rows_per_split, cudaStream_t stream);
 // vt[blk][j][k] = v[blk][k][j] for `blocks` blocks of b x c (KS values transposed per (i, l)).
 cudaError_t launch_transpose_blocks(const void *v, void *vt, int64_t blocks, int64_t b, int64_t c, int dtype,
                                     cudaStream_t stream);

@@ -150,6 +150,15 @@ def dv(dY, X, pattern) -> np.ndarray:
     return dV
 
 
+def bias_grad(dY) -> np.ndarray:
+    """Bias gradient of y = x K^T + bias: db[col] = sum_n dY[n][col] (the bias
+    is added to every row), summed in fp64; zeros for an empty batch."""
+    G = _f64(dY)
+    if G.ndim != 2:
+        raise ValueError("dY must be batch x width")
+    return G.sum(axis=0) if G.shape[0] else np.zeros(G.shape[1], dtype=np.float64)
+
+
 def densify(values, pattern) -> np.ndarray:
     """The dense (a*b*d, a*c*d) matrix K of one factor."""
     a, b, c, d = _check_pattern(pattern)

@@ -164,6 +164,14 @@ def test_injected_allocation_failure_is_reported_before_any_launch(lib, monkeypa
     assert lib.ks_workspace_info(ctypes.byref(n), None) == 0 and n.value == 0  # nothing was ever allocated
 
 
+def test_fma_rate_probe_validates_on_the_host(lib):
+    assert lib.ks_fma_rate_probe(None, 4, 16, None) == 1
+    assert lib.ks_fma_rate_probe(P, 0, 16, None) == 1
+    assert lib.ks_fma_rate_probe(P, 4, 24, None) == 1  # not a multiple of 16
+    assert b"multiple of 16" in lib.ks_last_error()
+    assert lib.ks_fma_rate_probe(P + 2, 4, 16, None) == 2
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(_lib, "_lib", None)

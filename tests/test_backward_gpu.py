@@ -100,6 +100,38 @@ def test_kslinear_layer_gradients(dtype):
     assert oracle.max_rel_err(layer.values.grad.cpu().reshape(-1), oracle.dv(G2, X2, p)) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("batch,width", [(1, 1), (63, 300), (1000, 1536), (25216, 384), (5, 4097)])
+def test_bias_grad_matches_oracle(dtype, batch, width):
+    g = torch.Generator().manual_seed(batch + width)
+    dy = torch.randn(batch, width, generator=g).to(dtype)
+    db = ks.bias_grad(dy.to(DEV))
+    ks.sync_status()
+    tol = 1e-5 if dtype == torch.float32 else 1e-2
+    assert oracle.max_rel_err(db.cpu(), oracle.bias_grad(dy)) <= tol
+
+
+def test_bias_grad_of_empty_batch_is_zero_and_deterministic():
+    z = ks.bias_grad(torch.zeros(0, 77, device=DEV))
+    assert torch.equal(z.cpu(), torch.zeros(77))
+    dy = torch.randn(9000, 1536, device=DEV)
+    assert torch.equal(ks.bias_grad(dy), ks.bias_grad(dy))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_kslinear_bias_gradient_runs_in_the_library(dtype):
+    p = (1, 64, 32, 4)
+    torch.manual_seed(2)
+    layer = ks.KSLinear(p, bias=True, dtype=dtype, device=DEV)
+    x = torch.randn(130, inputs.in_features(p), device=DEV).to(dtype)
+    y = layer(x)
+    g = torch.randn_like(y)
+    y.backward(g)
+    ks.sync_status()
+    tol = 1e-5 if dtype == torch.float32 else 1e-2
+    assert oracle.max_rel_err(layer.bias.grad.cpu(), oracle.bias_grad(g.cpu())) <= tol
+
+
 def test_kslinear_trains_toward_a_ks_target():
     # a few SGD steps on a realisable target must reduce the loss (a smoke test
     # of the whole training step on the GPU path)

@@ -145,3 +145,25 @@ def pins_pass(lib):
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_backward_pins_catch_planted_mistake(tmp_path, name):
     assert not pins_pass(build_mutant(tmp_path, name))
+
+
+def test_bias_grad_closed_forms_and_the_epilogue_derivative():
+    # ones: every column sums to the batch; row n = n + 1: batch (batch + 1) / 2
+    np.testing.assert_array_equal(oracle.bias_grad(np.ones((7, 3))), [7.0, 7.0, 7.0])
+    rows = np.arange(1, 11, dtype=float)[:, None] * np.ones((1, 4))
+    np.testing.assert_array_equal(oracle.bias_grad(rows), [55.0] * 4)
+    np.testing.assert_array_equal(oracle.bias_grad(np.zeros((0, 5))), np.zeros(5))
+    # db is the derivative of L(b) = <act-free epilogue(X, V, b), G> in b: L is
+    # linear in b, so L(b + t e_col) - L(b) = t db[col] exactly (t a power of two)
+    p = (2, 3, 4, 2)
+    rng = np.random.default_rng(3)
+    X = rng.integers(-3, 4, size=(5, 2 * 4 * 2)).astype(float)
+    V = rng.integers(-3, 4, size=2 * 3 * 4 * 2).astype(float)
+    G = rng.integers(-3, 4, size=(5, 2 * 3 * 2)).astype(float)
+    b = rng.integers(-3, 4, size=2 * 3 * 2).astype(float)
+    L = lambda bb: float(np.sum(oracle.matmul_epilogue(X, V, p, bb, "none") * G))
+    db = oracle.bias_grad(G)
+    for col in range(b.size):
+        e = np.zeros_like(b)
+        e[col] = 0.5
+        assert L(b + e) - L(b) == 0.5 * db[col]
