@@ -162,6 +162,10 @@ def workload_runs(name):
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "bf16", i) for i, p in enumerate(inputs.sweep_patterns())]
     if name == "sweep-tf32":
         return [(f"sweep[{i}]", p, inputs.SWEEP_BATCH, "tf32", i) for i, p in enumerate(inputs.sweep_patterns())]
+    if name == "sweep-sample":  # every 32nd pattern in both dtypes: the sample ncu's DRAM counters are taken on
+        pats = inputs.sweep_patterns()
+        return [(f"sweep[{i}]", pats[i], inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16")
+                for i in range(0, len(pats), 32)]
     if name == "sweep-quick":  # every 8th pattern, for development only
         pats = inputs.sweep_patterns()
         return [(f"sweep[{i}]", pats[i], inputs.SWEEP_BATCH, dt, i) for dt in ("fp32", "bf16")

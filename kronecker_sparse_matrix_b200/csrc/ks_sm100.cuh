@@ -202,6 +202,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t ss
                  "r"(x), "r"(y), "r"(ssrc)
                  : "memory");
 }
+// TMA tensor store of a 4-D box from shared memory (bulk group of this
+// thread); c0 is the innermost element coordinate (c0 * element size a
+// multiple of 16 bytes).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t ssrc, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(ssrc)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // this thread's bulk copies have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

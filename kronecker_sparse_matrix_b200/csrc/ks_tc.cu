@@ -45,8 +45,9 @@
 //               rows), convert to the storage type, interleave the l planes
 //               back into Y's (k, l) order in a shared-memory staging box of 32
 //               rows, and hand it to a TMA tensor store when the box is
-//               contiguous in Y (d == DLS), or copy it out in 16-byte stores
-//               otherwise.
+//               contiguous in Y (d == DLS); for fp32 with d > DLS, to a 4-D
+//               tensor store whose box is [k][row][l] (32-byte runs of Y);
+//               otherwise copy it out in 16-byte stores.
 //
 // TF32: the tensor core reads each fp32 operand at TF32 precision (10
 // explicit mantissa bits); products and sums are fp32.
@@ -135,7 +136,8 @@ struct TcParams {
     int v_stage_bytes;
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
     int box_row_bytes;               // staging row stride when not swizzled (an odd number of 16-byte units)
-    int ytma;                        // the swizzled staging box goes to Y as one TMA store (d == DLS)
+    int ytma;                        // 1: the staging box goes to Y as one 2-D TMA store (d == DLS);
+                                     // 2: as one 4-D store of a [k][row][l] box (fp32, d > DLS)
     int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
@@ -539,7 +541,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 w[h] = __float_as_uint(acc[f % DLS][f / DLS]);
                             }
                         }
-                        const uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
+                        uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
+                        // 4-D box (fp32 only): [k][row][l], unit u = (k, l0u .. l0u + RPU - 1); the
+                        // eight lanes of a 16-byte store reach at least four bank groups
+                        if (ES == 4 && p.ytma == 2)
+                            off = ((RPU * u) / DLS) * (32 * DLS * ES) + lane * (DLS * ES) + ((RPU * u) % DLS) * ES;
                         *reinterpret_cast<uint4 *>(stage + off) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
@@ -551,7 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async();
                     __syncwarp();
                     if (lane == 0 && (long long)row0 < p.N) {
-                        tma_store_2d(&ymap, su32(stage), (int)(ybase + (long long)kq * p.d), row0);
+                        if (ES == 4 && p.ytma == 2)
+                            tma_store_4d(&ymap, su32(stage), l0, row0, kq, i);
+                        else
+                            tma_store_2d(&ymap, su32(stage), (int)(ybase + (long long)kq * p.d), row0);
                         bulk_commit();
                     }
                     continue;
@@ -760,9 +769,24 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     if (kc == 0) return cudaErrorInvalidConfiguration;
     const int bi = DLS * kc;  // elements per staging row
     const bool sw128 = bi * ES == kChunkBytes;
-    const bool ytma = pr.d == DLS && (reinterpret_cast<uintptr_t>(pr.Y) % 16) == 0;
+    const bool yal = (reinterpret_cast<uintptr_t>(pr.Y) % 16) == 0;
+    const bool ytma = pr.d == DLS && yal;
+    // fp32 with d > DLS: Y viewed as (d, N, b, a), a box (DLS l, 32 rows, kc k,
+    // 1 block) whose shared image is [k][row][l] with 32-byte (k, row) runs and
+    // no swizzle.  (Measured against the 16-byte stores: 1.11x median on the
+    // d >= 16 TF32 patterns; for bf16 the 16-byte runs made it slower.)
+    const bool y4d = ES == 4 && pr.d > DLS && yal;
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
+    if (y4d) {
+        cuuint64_t dims[4] = {(cuuint64_t)pr.d, (cuuint64_t)pr.batch, (cuuint64_t)pr.b, (cuuint64_t)pr.a};
+        cuuint64_t strides[3] = {(cuuint64_t)pr.out_features() * ES, (cuuint64_t)pr.d * ES,
+                                 (cuuint64_t)pr.b * pr.d * ES};
+        cuuint32_t box[4] = {(cuuint32_t)DLS, 32, (cuuint32_t)kc, 1};
+        r = encode(&ymap, kType, 4, pr.Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     if (ytma) {
         // Y as (out_f, N): a box (DLS*kc elements, 32 rows); 128-byte rows with the
         // 128-byte swizzle of the staging, shorter rows packed densely
@@ -779,7 +803,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.box_elems = bi;
     p.box_sw128 = sw128 ? 1 : 0;
     p.box_row_bytes = bi * ES + ((bi * ES / 16) % 2 == 0 ? 16 : 0);
-    p.ytma = ytma ? 1 : 0;
+    p.ytma = ytma ? 1 : y4d ? 2 : 0;
     p.x3d = x3d ? 1 : 0;
     p.N = pr.batch;
     p.bias = pr.bias;

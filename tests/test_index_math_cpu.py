@@ -337,8 +337,9 @@ def tc_kc(dls, bp, es=2):
                                (1, 48, 8, 1), (2, 256, 64, 16)])
 def test_tc_epilogue_writes_each_output_once(p, es):
     """The output boxes of a tile: 32 rows x (DLS * kc) elements per warp and
-    chunk, either one tensor store of a contiguous box (d == DLS) or 16-byte
-    stores of its units; N = 300 leaves a ragged last row block."""
+    chunk, either one tensor store of a contiguous box (d == DLS), one 4-D
+    tensor store of a [k][row][l] box (fp32, d > DLS) or 16-byte stores of its
+    units; N = 300 leaves a ragged last row block."""
     a, b, c, d = p
     dls = 8 if d % 8 == 0 else d
     bp = tc_bp(dls, b)
@@ -366,6 +367,14 @@ def test_tc_epilogue_writes_each_output_once(p, es):
                                 for r in range(min(32, n - row0)):
                                     for e in range(dls * kc):
                                         written[(row0 + r, x + e)] += 1
+                            elif es == 4:  # one 4-D box [k][row][l] of Y viewed as (d, N, b, a)
+                                if row0 >= n:
+                                    continue
+                                assert (l0 * es) % 16 == 0 and kq + kc <= b
+                                for k in range(kc):
+                                    for r in range(min(32, n - row0)):
+                                        for l in range(dls):
+                                            written[(row0 + r, i * b * d + (kq + k) * d + l0 + l)] += 1
                             else:
                                 for lane in range(32):
                                     u = lane & 7
@@ -401,3 +410,32 @@ def test_tc_shared_memory_offsets_keep_their_alignment(dls, es):
             for vs in range(4):
                 for l in range(dls):
                     assert (off_v + vs * vstage + l * plane) % atom == 0
+
+
+@pytest.mark.parametrize("es", [2, 4])
+def test_tc_4d_store_staging_is_the_box_in_order(es):
+    """fp32 with d > DLS: the epilogue writes unit u of row `lane` at
+    ((RPU u) / DLS) * 32 DLS es + lane * DLS es + ((RPU u) % DLS) es, which must
+    be exactly the box (DLS l, 32 rows, kc k) in its shared order (l fastest,
+    then row, then k), every byte once, within the 4 KB staging; eight lanes of
+    one 16-byte store reach at least four bank groups.  (The bf16 form of this
+    layout is modelled too although bf16 keeps its 16-byte stores.)"""
+    dls, rpu = 8, 16 // es
+    kc = (128 // es) // dls
+    units = dls * kc * es // 16
+    seen = set()
+    for lane in range(32):
+        for u in range(units):
+            off = ((rpu * u) // dls) * (32 * dls * es) + lane * (dls * es) + ((rpu * u) % dls) * es
+            for h in range(rpu):
+                f = rpu * u + h
+                k, l = f // dls, f % dls
+                box = ((k * 32 + lane) * dls + l) * es
+                assert off + h * es == box and box not in seen
+                seen.add(box)
+    assert len(seen) == kc * 32 * dls and max(seen) + es <= 4096
+    for u in range(units):
+        for q0 in range(0, 32, 8):
+            g = [(((rpu * u) // dls) * (32 * dls * es) + lane * (dls * es) + ((rpu * u) % dls) * es) // 16 % 8
+                 for lane in range(q0, q0 + 8)]
+            assert max(g.count(x) for x in g) <= 2
