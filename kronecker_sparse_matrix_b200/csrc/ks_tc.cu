@@ -136,8 +136,8 @@ struct TcParams {
     int v_stage_bytes;
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
     int box_row_bytes;               // staging row stride when not swizzled (an odd number of 16-byte units)
-    int ytma;                        // 1: the staging box goes to Y as one 2-D TMA store (d == DLS);
-                                     // 2: as one 4-D store of a [k][row][l] box (fp32, d > DLS)
+    int ytma;                        // the staging box goes to Y as one TMA store: 2-D (d == DLS) or,
+                                     // in the Y4 kernels, 4-D ([k][row][l] box, fp32 with d > DLS)
     int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
@@ -160,7 +160,11 @@ __device__ __forceinline__ void transpose4x4_b32(const uint4 (&in)[4], uint4 (&o
     out[3] = make_uint4(in[0].w, in[1].w, in[2].w, in[3].w);
 }
 
-template <int DLS, typename T, bool EP>  // EP: fused bias / activation epilogue compiled in
+// EP: fused bias / activation epilogue compiled in; Y4: the output boxes go to
+// a 4-D TMA store of [k][row][l] boxes (fp32 with d > DLS), chosen at compile
+// time so that the other instantiations carry none of it (a run-time choice
+// cost the d == DLS TF32 epilogue 5-7%).
+template <int DLS, typename T, bool EP, bool Y4 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap vmap,
               const __grid_constant__ CUtensorMap ymap, const TcParams p) {
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
                         // 4-D box (fp32 only): [k][row][l], unit u = (k, l0u .. l0u + RPU - 1); the
                         // eight lanes of a 16-byte store reach at least four bank groups
-                        if (ES == 4 && p.ytma == 2)
+                        if constexpr (Y4)
                             off = ((RPU * u) / DLS) * (32 * DLS * ES) + lane * (DLS * ES) + ((RPU * u) % DLS) * ES;
                         *reinterpret_cast<uint4 *>(stage + off) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
@@ -557,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async();
                     __syncwarp();
                     if (lane == 0 && (long long)row0 < p.N) {
-                        if (ES == 4 && p.ytma == 2)
+                        if constexpr (Y4)
                             tma_store_4d(&ymap, su32(stage), l0, row0, kq, i);
                         else
                             tma_store_2d(&ymap, su32(stage), (int)(ybase + (long long)kq * p.d), row0);
@@ -775,7 +779,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     // 1 block) whose shared image is [k][row][l] with 32-byte (k, row) runs and
     // no swizzle.  (Measured against the 16-byte stores: 1.11x median on the
     // d >= 16 TF32 patterns; for bf16 the 16-byte runs made it slower.)
-    const bool y4d = ES == 4 && pr.d > DLS && yal;
+    const bool y4d = ES == 4 && DLS == 8 && pr.d > DLS && yal;
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
     if (y4d) {
@@ -829,7 +833,10 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.off_epi = L.off_epi;
     p.off_bar = L.off_bar;
     p.v_stage_bytes = L.v_stage_bytes;
-    auto kern = (pr.bias || pr.act) ? tc_kernel<DLS, T, true> : tc_kernel<DLS, T, false>;
+    const bool ep = pr.bias || pr.act;
+    auto kern = ep ? tc_kernel<DLS, T, true> : tc_kernel<DLS, T, false>;
+    if constexpr (ES == 4 && DLS == 8)
+        if (y4d) kern = ep ? tc_kernel<DLS, T, true, true> : tc_kernel<DLS, T, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (e != cudaSuccess) return e;
     const long long grid = std::min<long long>(p.n_tiles, (long long)sm_count());
