@@ -116,6 +116,24 @@ ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
                     int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
                     void *stream);
 
+/* ks_matmul for a batch that lives in HOST memory: X (batch x a*c*d),
+ * values and Y (batch x a*b*d) are HOST pointers, laid out as for ks_matmul.
+ * The library copies the values to the device once and streams the rows
+ * through in chunks (about six, each a multiple of 128 rows, at least 1024):
+ * the copy of chunk k+1 to the device, the product of chunk k and the copy of
+ * chunk k-1 back to the host run at the same time, on three streams the
+ * library keeps per device, ordered after earlier work on `stream`; `stream`
+ * waits for the whole call, which is asynchronous like every entry point
+ * (synchronise `stream` before reading Y or reusing X).  Page-locked host
+ * memory (cudaHostAlloc / cudaHostRegister) lets the copies overlap; pageable
+ * memory gives the same result without the overlap.  The device buffers (the
+ * values and two chunks of X and of Y) come from the library's pool, stream-
+ * ordered on `stream` (KS_ERR_ALLOC if that fails).  The product of each chunk
+ * is the one ks_matmul picks. */
+ks_status ks_matmul_host(const void *X, const void *values, int64_t a, int64_t b,
+                         int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
+                         void *stream);
+
 /* ks_matmul with a fused epilogue (the MLP shapes' bias and activation):
  *     Y[n][col] = act(sum_j ... + bias[col]),  col = i*b*d + k*d + l,
  * computed on the fp32 accumulator before the single rounding to the storage
@@ -123,7 +141,11 @@ ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
  * array of a*b*d elements of the storage dtype, or NULL for none; activation
  * is a ks_activation (other values: KS_ERR_INVALID_ARG).  bias must not
  * overlap Y.  variant is a ks_variant as for ks_matmul_variant.  With bias
- * NULL, KS_ACT_NONE and KS_VARIANT_AUTO this is ks_matmul. */
+ * NULL, KS_ACT_NONE and KS_VARIANT_AUTO this is ks_matmul.  The tensor-core
+ * kernel (KS_TF32, KS_BF16) takes a bias only if it is 16-byte aligned (else
+ * the CUDA-core kernel runs) and computes the tanh form of GELU with the
+ * hardware tanh approximation (relative error about 2^-11, far inside the
+ * TF32 and bf16 tolerances); KS_F32 products use CUDA's expf-based form. */
 ks_status ks_matmul_ep(const void *X, const void *values, int64_t a, int64_t b,
                        int64_t c, int64_t d, int64_t batch, void *Y, int dtype,
                        const void *bias, int activation, int variant,

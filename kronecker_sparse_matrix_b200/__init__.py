@@ -21,7 +21,7 @@ from ._lib import (KS_BF16, KS_F32, KS_TF32, KS_VARIANT_AUTO, KS_VARIANT_FMA,  #
 
 Pattern = Tuple[int, int, int, int]
 
-__all__ = ["matmul", "chain", "plan", "sync_status", "workspace_info", "ks_dtype_of", "KsError", "VARIANTS"]
+__all__ = ["matmul", "matmul_host", "chain", "plan", "sync_status", "workspace_info", "ks_dtype_of", "KsError", "VARIANTS"]
 
 
 def ks_dtype_of(t: torch.Tensor, tf32: bool = False) -> int:
@@ -71,6 +71,32 @@ def matmul(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Opti
     with torch.cuda.device(x.device):
         st = lib.ks_matmul_ep(x.data_ptr(), values.data_ptr(), a, b, c, d, batch, out.data_ptr(), dt, bias_ptr,
                               _act(act), _variant(variant), _stream_ptr(stream, x.device))
+    _lib.check(st)
+    return out
+
+
+def matmul_host(x: torch.Tensor, values: torch.Tensor, pattern: Pattern, *, out: Optional[torch.Tensor] = None,
+                tf32: bool = False, device: Optional[torch.device] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Y = X K^T for CPU tensors x (batch, a*c*d) and values, computed on the
+    GPU (``device``, default the current one) with the rows streamed through in
+    chunks whose copies overlap the products (pinned x, values and out give the
+    overlap).  Asynchronous on ``stream``: synchronise it before reading out."""
+    a, b, c, d = (int(v) for v in pattern)
+    if x.dim() != 2 or x.is_cuda or values.is_cuda:
+        raise ValueError("x must be a 2-D CPU tensor and values a CPU tensor")
+    if not (x.is_contiguous() and values.is_contiguous()) or values.dtype != x.dtype:
+        raise ValueError("x and values must be contiguous, with one dtype")
+    dt = ks_dtype_of(x, tf32)
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, a * b * d), dtype=x.dtype, pin_memory=x.is_pinned())
+    elif out.is_cuda or not out.is_contiguous() or out.dtype != x.dtype or out.shape != (batch, a * b * d):
+        raise ValueError("out must be a contiguous CPU tensor (batch, a*b*d) with x's dtype")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        st = _lib.load().ks_matmul_host(x.data_ptr(), values.data_ptr(), a, b, c, d, batch, out.data_ptr(), dt,
+                                        _stream_ptr(stream, dev))
     _lib.check(st)
     return out
 

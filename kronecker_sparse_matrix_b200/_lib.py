@@ -37,6 +37,7 @@ class KsPattern(ctypes.Structure):
 SIGNATURES = {
     "ks_matmul": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_matmul_variant": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp]),
+    "ks_matmul_host": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp]),
     "ks_plan": (_int, [_i64, _i64, _i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "ks_chain": (_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(KsPattern), _int, _i64, _vp, _int, _vp]),
     "ks_matmul_ep": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _int, _vp, _int, _int, _vp]),

@@ -464,6 +464,144 @@ ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b, int6
     return result == KS_OK ? ok() : result;
 }
 
+}  // extern "C"
+
+namespace ks {
+namespace {
+
+// Three non-blocking streams per device for ks_matmul_host: host-to-device
+// copies, products, device-to-host copies (created on first use, kept until
+// the process exits).
+cudaError_t host_streams(cudaStream_t (&out)[3]) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][3] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int k = 0; k < 3; ++k) {
+        if (!streams[dev][k]) {
+            e = cudaStreamCreateWithFlags(&streams[dev][k], cudaStreamNonBlocking);
+            if (e != cudaSuccess) return e;
+        }
+        out[k] = streams[dev][k];
+    }
+    return cudaSuccess;
+}
+
+// Rows per chunk of a host-resident product: about six chunks, each at least
+// 1024 rows and a multiple of 128 (the tensor-core tile), at most 256 MiB of
+// X plus Y per buffer.
+int64_t host_chunk_rows(int64_t batch, int64_t row_bytes) {
+    int64_t r = std::max<int64_t>(1024, (batch + 5) / 6);
+    r = (r + 127) / 128 * 128;
+    const int64_t cap = std::max<int64_t>(128, ((int64_t)256 << 20) / std::max<int64_t>(row_bytes, 1) / 128 * 128);
+    return std::min(std::min(r, cap), batch);
+}
+
+}  // namespace
+}  // namespace ks
+
+extern "C" {
+
+ks_status ks_matmul_host(const void *X, const void *values, int64_t a, int64_t b, int64_t c, int64_t d, int64_t batch,
+                         void *Y, int dtype, void *stream) {
+    ks_status s = check_dtype(dtype);
+    if (s != KS_OK) return s;
+    int64_t in_f = 0, out_f = 0, nvals = 0;
+    if ((s = check_sizes(a, b, c, d, batch, &in_f, &out_f, &nvals)) != KS_OK) return s;
+    if (batch == 0) return KS_OK;
+    if (!X || !values || !Y) return fail(KS_ERR_INVALID_ARG, "X, values and Y must be non-null");
+    const int elem = dtype == KS_BF16 ? 2 : 4;
+    if ((s = check_align(X, elem, "X")) != KS_OK || (s = check_align(values, elem, "values")) != KS_OK ||
+        (s = check_align(Y, elem, "Y")) != KS_OK)
+        return s;
+    const int64_t ybytes = batch * out_f * elem;
+    if (ranges_overlap(Y, ybytes, X, batch * in_f * elem)) return fail(KS_ERR_INVALID_ARG, "Y overlaps X");
+    if (ranges_overlap(Y, ybytes, values, nvals * elem)) return fail(KS_ERR_INVALID_ARG, "Y overlaps values");
+    cudaStream_t caller = static_cast<cudaStream_t>(stream);
+    cudaStream_t st[3];
+    cudaError_t e = host_streams(st);
+    if (e != cudaSuccess) return cuda_fail(e, "creating the copy and product streams");
+    const int64_t rows = host_chunk_rows(batch, (in_f + out_f) * elem);
+    const int64_t n_chunks = (batch + rows - 1) / rows;
+    const int nbuf = n_chunks > 1 ? 2 : 1;
+    const size_t vbytes = ((size_t)(nvals * elem) + 255) / 256 * 256;
+    const size_t xb = ((size_t)(rows * in_f * elem) + 255) / 256 * 256;
+    const size_t yb = ((size_t)(rows * out_f * elem) + 255) / 256 * 256;
+    char *dev = nullptr;
+    e = pool_alloc(reinterpret_cast<void **>(&dev), vbytes + nbuf * (xb + yb), caller);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(KS_ERR_ALLOC, "workspace allocation of %zu bytes failed: %s", vbytes + nbuf * (xb + yb),
+                    cudaGetErrorString(e));
+    }
+    char *dv = dev, *dx[2] = {dev + vbytes, dev + vbytes + xb}, *dy[2] = {dev + vbytes + nbuf * xb,
+                                                                         dev + vbytes + nbuf * xb + yb};
+    // events: fork, and per buffer the last copy-in, product and copy-out on it
+    cudaEvent_t ev[8] = {};
+    ks_status result = KS_OK;
+    for (int k = 0; k < 8 && result == KS_OK; ++k)
+        if ((e = cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming)) != cudaSuccess)
+            result = cuda_fail(e, "event create");
+    cudaEvent_t fork = ev[0], vin = ev[1], in_done[2] = {ev[2], ev[3]}, cmp_done[2] = {ev[4], ev[5]},
+                out_done[2] = {ev[6], ev[7]};
+    auto chk = [&](cudaError_t err, const char *what) {
+        if (err != cudaSuccess && result == KS_OK) result = cuda_fail(err, what);
+        return result == KS_OK;
+    };
+    if (result == KS_OK && chk(cudaEventRecord(fork, caller), "event record")) {
+        for (int k = 0; k < 3; ++k) chk(cudaStreamWaitEvent(st[k], fork, 0), "stream wait");
+        chk(cudaMemcpyAsync(dv, values, (size_t)(nvals * elem), cudaMemcpyHostToDevice, st[0]), "values copy");
+        chk(cudaEventRecord(vin, st[0]), "event record");
+        chk(cudaStreamWaitEvent(st[1], vin, 0), "stream wait");
+    }
+    for (int64_t k = 0; k < n_chunks && result == KS_OK; ++k) {
+        const int q = (int)(k % nbuf);
+        const int64_t r0 = k * rows, nr = std::min(rows, batch - r0);
+        // copy-in: the product of chunk k - 2 has finished reading dx[q]
+        if (k >= nbuf) chk(cudaStreamWaitEvent(st[0], cmp_done[q], 0), "stream wait");
+        chk(cudaMemcpyAsync(dx[q], static_cast<const char *>(X) + r0 * in_f * elem, (size_t)(nr * in_f * elem),
+                            cudaMemcpyHostToDevice, st[0]),
+            "X copy");
+        chk(cudaEventRecord(in_done[q], st[0]), "event record");
+        // product: its X has landed and the copy-out of chunk k - 2 has read dy[q]
+        chk(cudaStreamWaitEvent(st[1], in_done[q], 0), "stream wait");
+        if (k >= nbuf) chk(cudaStreamWaitEvent(st[1], out_done[q], 0), "stream wait");
+        if (result != KS_OK) break;
+        Problem p{dx[q], dv, dy[q], a, b, c, d, nr, dtype, st[1]};
+        const ks_status r = run(p, KS_VARIANT_AUTO);
+        if (r != KS_OK) {
+            result = r;
+            break;
+        }
+        chk(cudaEventRecord(cmp_done[q], st[1]), "event record");
+        // copy-out
+        chk(cudaStreamWaitEvent(st[2], cmp_done[q], 0), "stream wait");
+        chk(cudaMemcpyAsync(static_cast<char *>(Y) + r0 * out_f * elem, dy[q], (size_t)(nr * out_f * elem),
+                            cudaMemcpyDeviceToHost, st[2]),
+            "Y copy");
+        chk(cudaEventRecord(out_done[q], st[2]), "event record");
+    }
+    // join: the caller's stream waits for all three streams, then frees the workspace
+    for (int k = 0; k < 3; ++k) {
+        cudaEvent_t j = nullptr;
+        if (cudaEventCreateWithFlags(&j, cudaEventDisableTiming) == cudaSuccess) {
+            if (cudaEventRecord(j, st[k]) == cudaSuccess) (void)cudaStreamWaitEvent(caller, j, 0);
+            (void)cudaEventDestroy(j);
+        } else {
+            (void)cudaGetLastError();
+            (void)cudaStreamSynchronize(st[k]);
+        }
+    }
+    e = cudaFreeAsync(dev, caller);
+    if (e != cudaSuccess && result == KS_OK) result = cuda_fail(e, "workspace free");
+    for (int k = 0; k < 8; ++k)
+        if (ev[k]) (void)cudaEventDestroy(ev[k]);
+    return result == KS_OK ? ok() : result;
+}
+
 ks_status ks_bias_grad(const void *dY, int64_t batch, int64_t width, void *db, int dtype, void *stream) {
     ks_status s = check_dtype(dtype);
     if (s != KS_OK) return s;

@@ -26,6 +26,19 @@ __device__ __forceinline__ float gelu_tanh_f(float z) {
     return 0.5f * z * (1.f + t);
 }
 
+// GELU, tanh form, with the hardware tanh approximation (tanh.approx.f32,
+// relative error about 2^-11): for the tensor-core outputs, whose tolerance
+// (bf16 rounding, TF32 operands) is far coarser than that.
+__device__ __forceinline__ float tanh_hw(float u) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(u));
+    return t;
+}
+__device__ __forceinline__ float gelu_tanh_hw(float z) {
+    const float u = 0.7978845608028654f * fmaf(0.044715f * z, z * z, z);
+    return 0.5f * z * (1.f + tanh_hw(u));
+}
+
 // GELU, erf form: z Phi(z) = z (1 + erf(z / sqrt 2)) / 2, CUDA's erff.
 __device__ __forceinline__ float gelu_erf_f(float z) { return 0.5f * z * (1.f + erff(z * 0.7071067811865476f)); }
 
@@ -57,6 +70,18 @@ __device__ __forceinline__ void ep_act_array(float (&v)[N], int act) {
             for (int e = 0; e < N; ++e) v[e] = gelu_erf_f(v[e]);
             break;
         default: break;
+    }
+}
+
+// ep_act_array with the hardware tanh for the tanh form of GELU (tensor-core
+// epilogues only).
+template <int N>
+__device__ __forceinline__ void ep_act_array_hw(float (&v)[N], int act) {
+    if (act == 2) {
+#pragma unroll
+        for (int e = 0; e < N; ++e) v[e] = gelu_tanh_hw(v[e]);
+    } else {
+        ep_act_array(v, act);
     }
 }
 

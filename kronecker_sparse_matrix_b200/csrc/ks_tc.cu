@@ -515,16 +515,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const int kq = ps * p.bp + oc * kc;  // first k of the chunk
                 const long long ybase = (long long)i * p.b * p.d + l0;
-                if (EP && bias) {  // fused epilogue on (k = kq + e, l)
+                if (EP && bias) {
+                    // fused epilogue on (k = kq + e, l): the chunk's bias in 16-byte units of
+                    // RPU consecutive l of one k (the same for every lane: one transaction each)
 #pragma unroll
-                    for (int l = 0; l < DLS; ++l)
+                    for (int u = 0; u < CE / RPU; ++u) {
+                        if (u < units) {
+                            const int e0 = (RPU * u) / DLS, lu = (RPU * u) % DLS;
+                            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(bias + ybase +
+                                                                                  (long long)(kq + e0) * p.d + lu));
+                            float bb[RPU];
+                            if constexpr (ES == 2) {
+                                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                        for (int e = 0; e < KCM; ++e)
-                            if (e < kc) acc[l][e] += ep_bias(bias, ybase + (long long)(kq + e) * p.d + l);
+                                for (int h = 0; h < 4; ++h) {
+                                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ww[h]));
+                                    bb[2 * h] = f2.x;
+                                    bb[2 * h + 1] = f2.y;
+                                }
+                            } else {
+                                bb[0] = __uint_as_float(w.x);
+                                bb[1] = __uint_as_float(w.y);
+                                bb[2] = __uint_as_float(w.z);
+                                bb[3] = __uint_as_float(w.w);
+                            }
+#pragma unroll
+                            for (int h = 0; h < RPU; ++h) {
+                                const int f = RPU * u + h;
+                                acc[f % DLS][f / DLS] += bb[h];
+                            }
+                        }
+                    }
                 }
                 if (EP && p.act) {
 #pragma unroll
-                    for (int l = 0; l < DLS; ++l) ep_act_array(acc[l], p.act);
+                    for (int l = 0; l < DLS; ++l) ep_act_array_hw(acc[l], p.act);
                 }
                 if (p.ytma) {  // the previous box store has finished reading the staging
                     if (lane == 0) bulk_wait_read_all();
@@ -710,6 +735,7 @@ bool tc_supported(const Problem &p, const char **why) {
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.X) | reinterpret_cast<uintptr_t>(p.V) |
                          reinterpret_cast<uintptr_t>(p.Y);
     if (al % 16) { *why = "X, values and Y must be 16-byte aligned"; return false; }
+    if (reinterpret_cast<uintptr_t>(p.bias) % 16) { *why = "a fused bias must be 16-byte aligned"; return false; }
     const int bp = tc_bp(dls, p.b);
     TcLayout L;
     if (bp == 0 || tc_kc(dls, bp, es) == 0) { *why = "b has no pass width (a multiple of 16 dividing it)"; return false; }

@@ -151,6 +151,8 @@ def test_tc_variant_refuses_fp32(lib):
 
 
 def test_injected_allocation_failure_is_reported_before_any_launch(lib, monkeypatch):
+    n0 = ctypes.c_int64(-1)
+    assert lib.ks_workspace_info(ctypes.byref(n0), None) == 0
     monkeypatch.setenv("KS_FAULT_INJECT", "alloc")
     pats = (_lib.KsPattern * 2)(_lib.KsPattern(1, 4, 4, 2), _lib.KsPattern(2, 4, 4, 1))
     ptrs = (ctypes.c_void_p * 2)(P * 2, P * 3)
@@ -161,7 +163,15 @@ def test_injected_allocation_failure_is_reported_before_any_launch(lib, monkeypa
     facs = (ctypes.c_void_p * 4)(P * 4, P * 5, P * 6, P * 7)
     assert lib.ks_butterfly_factorize(P, 4, facs, 0, None) == 4
     n = ctypes.c_int64(-1)
-    assert lib.ks_workspace_info(ctypes.byref(n), None) == 0 and n.value == 0  # nothing was ever allocated
+    assert lib.ks_workspace_info(ctypes.byref(n), None) == 0 and n.value == n0.value  # nothing was allocated
+
+
+def test_host_product_validates_on_the_host(lib):
+    assert lib.ks_matmul_host(None, P, 2, 2, 2, 2, 4, P * 8, 0, None) == 1
+    assert lib.ks_matmul_host(P, P, 2, 2, 2, 2, 4, P, 0, None) == 1  # Y overlaps X
+    assert b"overlaps X" in lib.ks_last_error()
+    assert lib.ks_matmul_host(P + 2, P * 4, 2, 2, 2, 2, 4, P * 8, 0, None) == 2
+    assert lib.ks_matmul_host(None, None, 2, 2, 2, 2, 0, None, 0, None) == 0  # batch 0: no-op
 
 
 def test_fma_rate_probe_validates_on_the_host(lib):

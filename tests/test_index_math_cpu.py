@@ -439,3 +439,38 @@ def test_tc_4d_store_staging_is_the_box_in_order(es):
             g = [(((rpu * u) // dls) * (32 * dls * es) + lane * (dls * es) + ((rpu * u) % dls) * es) // 16 % 8
                  for lane in range(q0, q0 + 8)]
             assert max(g.count(x) for x in g) <= 2
+
+
+@pytest.mark.parametrize("es", [2, 4])
+def test_tc_fused_bias_units_are_aligned_and_cover_the_chunk(es):
+    """The tensor-core epilogue reads a chunk's bias as 16-byte units of RPU
+    consecutive (k, l) outputs at bias + ybase + (kq + e0) * d + lu: every unit
+    is 16-byte aligned (for a 16-byte-aligned bias) and the units cover the
+    chunk's kc x DLS columns exactly once, on sweep and test patterns."""
+    from kronecker_sparse_matrix_b200 import inputs
+    pats = inputs.sweep_patterns()[::5] + [(1, 192, 48, 8), (1, 256, 64, 16), (2, 64, 64, 2), (4, 64, 32, 1),
+                                           (2, 48, 24, 2), (1, 32, 40, 4), (1, 16, 56, 8), (3, 32, 16, 4),
+                                           (2, 64, 64, 32), (1, 48, 48, 1), (1, 64, 8, 1)]
+    rpu = 16 // es
+    for (a, b, c, d) in pats:
+        if c % (32 // es):
+            continue
+        dls = 8 if d % 8 == 0 else d
+        bp = tc_bp(dls, b)
+        kc = tc_kc(dls, bp, es) if bp else 0
+        if not kc:
+            continue
+        units = dls * kc * es // 16
+        for i in range(min(a, 2)):
+            for l0 in range(0, d, dls):
+                ybase = i * b * d + l0
+                for kq in range(0, b, kc):
+                    cols = []
+                    for u in range(units):
+                        e0, lu = (rpu * u) // dls, (rpu * u) % dls
+                        off = ybase + (kq + e0) * d + lu
+                        assert (off * es) % 16 == 0
+                        cols += [off + h for h in range(rpu)]
+                        assert all(off + h == ybase + (kq + (rpu * u + h) // dls) * d + (rpu * u + h) % dls
+                                   for h in range(rpu))
+                    assert sorted(cols) == sorted(ybase + (kq + e) * d + l for e in range(kc) for l in range(dls))
