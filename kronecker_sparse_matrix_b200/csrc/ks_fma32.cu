@@ -14,7 +14,9 @@
 // lanes and leave straight from registers: no shared-memory interleave of
 // the l, no barrier after a tile.  Operands reach shared memory without passing
 // through registers, in a ring of stages of 8 j whose copies run ahead of the
-// compute, across tile boundaries too:
+// compute, across tile boundaries too.  A warpgroup of its own (warps 8-11)
+// issues the copies; the eight compute warps (0-7) meet it only at each
+// stage's full and empty mbarriers:
 //
 //   X       16-byte cp.async of whole row segments, kept in X's own order:
 //           As[n][j*DL + l], row stride RA chosen so that one warp's loads
@@ -36,14 +38,17 @@
 
 #include "ks_epilogue.cuh"
 #include "ks_internal.h"
+#include "ks_sm100.cuh"
 
 namespace ks {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kJT = 8;   // j per stage
+constexpr int kThreads = 384;    // eight compute warps, then a copy-issuing warpgroup
+constexpr int kCopyRoles = 256;  // copy roles per stage (two per copy thread)
+constexpr int kJT = 8;           // j per stage
 
 struct Fma32Params {
+    unsigned *status;
     const float *X;
     const float *V;
     float *Y;
@@ -88,8 +93,7 @@ struct Tile32 {
     static constexpr int NS = (DL == 4 && 4 * STAGE * 4 <= 232448) ? 4 : 3;
     static constexpr int SMEM_FLOATS = NS * STAGE;
     static constexpr int CA = 2 * DL;                 // 16-byte chunks per A row per stage
-    static constexpr int NXC = (BM * CA + kThreads - 1) / kThreads;      // A copies per thread
-    static constexpr int NV = (DL * BKL * kJT + kThreads - 1) / kThreads;  // values copies per thread
+    static constexpr int NXC = (BM * CA + kCopyRoles - 1) / kCopyRoles;  // A copies per role
 };
 
 // Fused bias and activation of four consecutive outputs (columns col..col+3).
@@ -119,13 +123,28 @@ __device__ __forceinline__ void cp_async16_full(uint32_t dst, const float *src) 
 __device__ __forceinline__ void cp_async4_full(uint32_t dst, const float *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// The mbarrier receives one arrival when every cp.async this thread issued
+// before it has landed (.noinc: that arrival is one of the barrier's expected
+// count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(sm100::su32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // VT: p.V holds the values transposed per block, vt[i][l][j][k] (k
 // contiguous), and goes to shared memory with 16-byte copies; otherwise the
 // values keep their [i][l][k][j] layout and move as 4-byte transposing copies.
+//
+// Warps 8-11 issue every copy: each of their 128 threads plays two of the
+// stage's 256 copy roles and signals the stage's full barrier when its copies
+// have landed (cp.async.mbarrier.arrive.noinc, 128 arrivals per phase).  Warps
+// 0-7 only compute: they wait for full stages and release them through the
+// empty barriers (one arrival per warp), so warps drift apart and one warp's
+// epilogue overlaps the others' products; no CTA-wide barrier runs after the
+// start.  The copy warpgroup gives registers to the compute warps
+// (setmaxnreg: 128 x 40 + 256 x 232 = the 384 x 168 of the launch).  Every
+// wait is bounded; a wait that runs out sets the device status word and the
+// CTA's abort flag, which ends every role's loop.
 template <int DL, int WM, int WK, int TN, bool VT>
 __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p) {
     using TL = Tile32<DL, WM, WK, TN>;
@@ -133,164 +152,154 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
     using LN = typename TL::LN;
     extern __shared__ __align__(16) float smem[];
     constexpr int kNS = TL::NS;
+    constexpr int kBarOff = (TL::SMEM_FLOATS * 4 + 15) / 16 * 16;  // bytes
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(smem) + kBarOff);
+    uint64_t *empty_bar = full_bar + kNS;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + kNS);
     const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(smem);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int w_m = warp / WK;
-    const int w_k = warp % WK;
-    // compute roles: lane = (row group, l, k group), k group fastest
-    const int c_kq = lane % LN::KQ, c_l = (lane / LN::KQ) % DL, c_rg = lane / (LN::KQ * DL);
     const int groups_per_i = p.d / DL;
     const int S = p.n_stages;
     const int my_tiles = (p.n_tiles > (int)blockIdx.x) ? (p.n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 
-    // Per-thread copy roles, fixed for the whole kernel.
-    //   X: chunk q = tid % CA of rows tid / CA + t * XR (t < NXC): elements
-    //      f = 4q..4q+3 of the row's (j * DL + l), i.e. j = jx, l = lx..lx+3.
-    //   values: j = vj, k = kq + (32 t) % BKL, l = (32 t) / BKL (t < NV).
-    constexpr int XR = kThreads / TL::CA;
-    const int xn = tid / TL::CA, xf = 4 * (tid % TL::CA);
-    const int jx = xf / DL, lx = xf % DL;
-    const int vj = lane & 7, kq = tid >> 3;
-    const long long x_row_step = (long long)XR * p.in_f;
-    // VT copies: element e = tid + 256 t of the stage's (l, j, 4-k group), k fastest
-    constexpr int K4 = BKL / 4, NVT = (DL * kJT * K4 + kThreads - 1) / kThreads;
-
-    // Copy state: the next stage to issue is stage iss_s of tile iteration iss_it.
-    int iss_it = 0, iss_s = 0, iss_buf = 0;
-    const float *x_thr = p.X;  // this thread's first X chunk of the tile, at j = 0
-    const float *v_thr = p.V;  // values[i][l0][k0 + kq][vj] (VT: vt[i][l0][0][k0])
-    int x_rows = 0;            // rows left from this thread's first copy row
-    int k_left = 0;            // p.b - k0 - kq
-    bool full = false;         // every row and every k of the tile in range
-    auto set_issue_tile = [&](int it) {
-        const int tile = (int)blockIdx.x + it * (int)gridDim.x;
-        const int kb = tile % p.n_kb;
-        const int rest = tile / p.n_kb;
-        const int gg = rest % p.n_g;
-        const long long n0 = (long long)(rest / p.n_g) * BM;
-        const int i = gg / groups_per_i, l0 = (gg % groups_per_i) * DL;
-        const int k0 = kb * BKL;
-        x_rows = (int)min((long long)(BM + 1), p.N - n0) - xn;
-        k_left = p.b - k0 - kq;
-        full = (n0 + BM <= p.N) && (k0 + BKL <= p.b);
-        x_thr = p.X + (n0 + xn) * p.in_f + (long long)i * p.c * p.d + (long long)jx * p.d + l0 + lx;
-        if constexpr (VT)
-            v_thr = p.V + (long long)(i * p.d + l0) * p.c * p.b + k0;
-        else
-            v_thr = p.V + ((long long)(i * p.d + l0) * p.b + k0 + kq) * p.c + vj;
-    };
-    if (my_tiles > 0) set_issue_tile(0);
-
-    // values copy t: l = lt(t), k = kq + kt(t); its source offset from v_thr
-    auto v_lk = [&](int t, int &l, int &kc) {
-        if constexpr (BKL % 32 == 0) {
-            kc = (32 * t) % BKL;
-            l = (32 * t) / BKL;
-        } else {  // e = kq + 32 t split at runtime (BKL not a multiple of 32)
-            const int e8 = kq + 32 * t;
-            l = e8 / BKL;
-            kc = e8 % BKL - kq;
+    if (tid == 0) {
+        for (int s = 0; s < kNS; ++s) {
+            sm100::mbar_init(&full_bar[s], 128);
+            sm100::mbar_init(&empty_bar[s], 8);
         }
-    };
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
 
-    // Issues the copies of the next stage (if any is left) and commits a group.
-    auto issue = [&]() {
-        if (iss_it < my_tiles) {
-            const int j0 = iss_s * kJT;
-            const uint32_t st = s_base + (uint32_t)(iss_buf * TL::STAGE) * 4u;
-            const uint32_t sx = st + (uint32_t)(xn * TL::RA + xf) * 4u;
-            const uint32_t sv = st + (uint32_t)(TL::A_WORDS + vj * TL::BKP + kq) * 4u;
-            const float *xs = x_thr + (long long)j0 * p.d;
-            const float *vs = v_thr + j0;
-            if (full && j0 + kJT <= p.c) {
+    if (warp >= 8) {
+        // ------------------------------------------------ copy issue (warps 8-11, two copy roles per thread)
+        // registers: 256 x 232 + 128 x 40 = 64512 = 384 threads x 168 at launch
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+        const int pt = threadIdx.x - 256;  // 0..127
+        constexpr int kT = kCopyRoles;
+        constexpr int XR = kT / TL::CA;
+        constexpr int K4 = BKL / 4, NVT = (DL * kJT * K4 + kT - 1) / kT;
+        constexpr int NV = (DL * BKL * kJT + kT - 1) / kT;
+        const long long x_row_step = (long long)XR * p.in_f;
+        uint32_t fill = 0;
+        bool ok = true;
+        for (int it = 0; it < my_tiles && ok; ++it) {
+            const int tile = (int)blockIdx.x + it * (int)gridDim.x;
+            const int kb = tile % p.n_kb;
+            const int rest = tile / p.n_kb;
+            const int gg = rest % p.n_g;
+            const long long n0 = (long long)(rest / p.n_g) * BM;
+            const int i = gg / groups_per_i, l0 = (gg % groups_per_i) * DL;
+            const int k0 = kb * BKL;
+            const bool full_t = (n0 + BM <= p.N) && (k0 + BKL <= p.b);
+            for (int s = 0; s < S && ok; ++s, ++fill) {
+                const int buf = (int)(fill % kNS);
+                ok = sm100::mbar_wait(&empty_bar[buf], ((fill / kNS) & 1) ^ 1, abort_flag, p.status);
+                if (!ok) break;
+                const int j0 = s * kJT;
+                const uint32_t st = s_base + (uint32_t)(buf * TL::STAGE) * 4u;
+                const bool fast = full_t && j0 + kJT <= p.c;
+#pragma unroll 1
+                for (int v = 0; v < kT / (kThreads - 256); ++v) {
+                    const int vt = pt + 128 * v;
+                    const int xn = vt / TL::CA, xf = 4 * (vt % TL::CA);
+                    const int jx = xf / DL, lx = xf % DL;
+                    const int vj = vt & 7, kq = vt >> 3;
+                    const float *xs = p.X + (n0 + xn) * p.in_f + (long long)i * p.c * p.d + (long long)(j0 + jx) * p.d +
+                                      l0 + lx;
+                    const uint32_t sx = st + (uint32_t)(xn * TL::RA + xf) * 4u;
+                    const int x_rows = (int)min((long long)(BM + 1), p.N - n0) - xn;
+                    const bool jxv = j0 + jx < p.c;
 #pragma unroll
-                for (int t = 0; t < TL::NXC; ++t)
-                    if (TL::NXC * kThreads == BM * TL::CA || xn + t * XR < BM)
-                        cp_async16_full(sx + (uint32_t)(t * XR * TL::RA) * 4u, xs + t * x_row_step);
-                if constexpr (VT) {
-#pragma unroll
-                    for (int t = 0; t < NVT; ++t) {
-                        const int e = tid + t * kThreads;
-                        if (NVT * kThreads == DL * kJT * K4 || e < DL * kJT * K4) {
-                            const int k4 = e % K4, jl = e / K4, j = jl % kJT, l = jl / kJT;
-                            cp_async16_full(st + (uint32_t)(TL::A_WORDS + l * TL::PSB + j * TL::BKP + 4 * k4) * 4u,
-                                            v_thr + ((long long)(l * p.c + j0 + j) * p.b + 4 * k4));
+                    for (int t = 0; t < TL::NXC; ++t) {
+                        if (TL::NXC * kT == BM * TL::CA || xn + t * XR < BM) {
+                            if (fast) {
+                                cp_async16_full(sx + (uint32_t)(t * XR * TL::RA) * 4u, xs + t * x_row_step);
+                            } else {
+                                const bool ok2 = jxv && t * XR < x_rows;
+                                cp_async16(sx + (uint32_t)(t * XR * TL::RA) * 4u, ok2 ? xs + t * x_row_step : p.X, ok2);
+                            }
                         }
                     }
-                } else {
+                    if constexpr (VT) {
+                        const float *vbase = p.V + (long long)(i * p.d + l0) * p.c * p.b + k0;
 #pragma unroll
-                    for (int t = 0; t < TL::NV; ++t) {
-                        int l, kc;
-                        v_lk(t, l, kc);
-                        if (BKL % 32 == 0 || TL::NV * kThreads == DL * BKL * kJT || kq + 32 * t < DL * BKL)
-                            cp_async4_full(sv + (uint32_t)(l * TL::PSB + kc) * 4u, vs + (l * p.bc + kc * p.c));
-                    }
-                }
-            } else {
-                const bool jxv = j0 + jx < p.c;
+                        for (int t = 0; t < NVT; ++t) {
+                            const int e = vt + t * kT;
+                            if (NVT * kT == DL * kJT * K4 || e < DL * kJT * K4) {
+                                const int k4 = e % K4, jl = e / K4, j = jl % kJT, l = jl / kJT;
+                                const uint32_t dst = st + (uint32_t)(TL::A_WORDS + l * TL::PSB + j * TL::BKP + 4 * k4) * 4u;
+                                const float *src = vbase + ((long long)(l * p.c + j0 + j) * p.b + 4 * k4);
+                                if (fast) {
+                                    cp_async16_full(dst, src);
+                                } else {
+                                    const bool ok2 = (j0 + j < p.c) && (4 * k4 < p.b - k0);
+                                    cp_async16(dst, ok2 ? src : p.V, ok2);
+                                }
+                            }
+                        }
+                    } else {
+                        const float *vs = p.V + ((long long)(i * p.d + l0) * p.b + k0 + kq) * p.c + vj + j0;
+                        const uint32_t sv = st + (uint32_t)(TL::A_WORDS + vj * TL::BKP + kq) * 4u;
+                        const int k_left = p.b - k0 - kq;
+                        const bool jvv = j0 + vj < p.c;
 #pragma unroll
-                for (int t = 0; t < TL::NXC; ++t) {
-                    if (TL::NXC * kThreads == BM * TL::CA || xn + t * XR < BM) {
-                        const bool v = jxv && t * XR < x_rows;
-                        cp_async16(sx + (uint32_t)(t * XR * TL::RA) * 4u, v ? xs + t * x_row_step : p.X, v);
-                    }
-                }
-                if constexpr (VT) {
-#pragma unroll
-                    for (int t = 0; t < NVT; ++t) {
-                        const int e = tid + t * kThreads;
-                        if (NVT * kThreads == DL * kJT * K4 || e < DL * kJT * K4) {
-                            const int k4 = e % K4, jl = e / K4, j = jl % kJT, l = jl / kJT;
-                            const bool v = (j0 + j < p.c) && (4 * k4 < k_left + kq);  // k_left + kq = b - k0
-                            cp_async16(st + (uint32_t)(TL::A_WORDS + l * TL::PSB + j * TL::BKP + 4 * k4) * 4u,
-                                       v ? v_thr + ((long long)(l * p.c + j0 + j) * p.b + 4 * k4) : p.V, v);
+                        for (int t = 0; t < NV; ++t) {
+                            int l, kc;
+                            if constexpr (BKL % 32 == 0) {
+                                kc = (32 * t) % BKL;
+                                l = (32 * t) / BKL;
+                            } else {
+                                const int e8 = kq + 32 * t;
+                                l = e8 / BKL;
+                                kc = e8 % BKL - kq;
+                            }
+                            if (BKL % 32 == 0 || NV * kT == DL * BKL * kJT || kq + 32 * t < DL * BKL) {
+                                if (fast) {
+                                    cp_async4_full(sv + (uint32_t)(l * TL::PSB + kc) * 4u, vs + (l * p.bc + kc * p.c));
+                                } else {
+                                    const bool ok2 = jvv && kc < k_left;
+                                    cp_async4(sv + (uint32_t)(l * TL::PSB + kc) * 4u, ok2 ? vs + (l * p.bc + kc * p.c) : p.V,
+                                              ok2);
+                                }
+                            }
                         }
                     }
-                } else {
-                    const bool jvv = j0 + vj < p.c;
-#pragma unroll
-                    for (int t = 0; t < TL::NV; ++t) {
-                        int l, kc;
-                        v_lk(t, l, kc);
-                        if (BKL % 32 == 0 || TL::NV * kThreads == DL * BKL * kJT || kq + 32 * t < DL * BKL) {
-                            const bool v = jvv && kc < k_left;
-                            cp_async4(sv + (uint32_t)(l * TL::PSB + kc) * 4u, v ? vs + (l * p.bc + kc * p.c) : p.V, v);
-                        }
-                    }
                 }
-            }
-            if (++iss_s == S) {
-                iss_s = 0;
-                if (++iss_it < my_tiles) set_issue_tile(iss_it);
+                cp_async_mbar_arrive_noinc(&full_bar[buf]);  // fires when this lane's copies have landed
             }
         }
-        iss_buf = (iss_buf + 1 == kNS) ? 0 : iss_buf + 1;
-        cp_async_commit();  // one group per stage, empty or not
-    };
+        cp_async_wait_all();  // no copy may still be landing when the CTA exits
+        return;
+    }
 
-#pragma unroll
-    for (int g = 0; g < kNS - 1; ++g) issue();
-
+    // ------------------------------------------------ compute warps 0-7
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+    const int w_m = warp / WK;
+    const int w_k = warp % WK;
+    // compute roles: lane = (row group, l, k group), k group fastest
+    const int c_kq = lane % LN::KQ, c_l = (lane / LN::KQ) % DL, c_rg = lane / (LN::KQ * DL);
     // acc[m][2q + h]: row a_row + RG*m, k = b_col + 4*KQ*q + 2h + (0, 1), l = l0 + c_l
     float2 acc[8][TN / 2];
-    int buf = 0;  // ring buffer of the stage being computed
     const int a_row = w_m * (8 * LN::RG) + c_rg;
     const int b_col = w_k * TL::KW + 4 * c_kq;
-    for (int it = 0; it < my_tiles; ++it) {
+    uint32_t fill = 0;
+    bool ok = true;
+    for (int it = 0; it < my_tiles && ok; ++it) {
         const int tile = (int)blockIdx.x + it * (int)gridDim.x;
 #pragma unroll
         for (int m = 0; m < 8; ++m)
 #pragma unroll
             for (int kk = 0; kk < TN / 2; ++kk) acc[m][kk] = make_float2(0.f, 0.f);
 
-        for (int s = 0; s < S; ++s) {
-            cp_async_wait<kNS - 2>();
-            __syncthreads();
-            issue();  // into the buffer computed one step ago
+        for (int s = 0; s < S; ++s, ++fill) {
+            const int buf = (int)(fill % kNS);
+            ok = __all_sync(0xffffffffu, sm100::mbar_wait(&full_bar[buf], (fill / kNS) & 1, abort_flag, p.status));
+            if (!ok) break;
             const float *stage = smem + buf * TL::STAGE;
-            buf = (buf + 1 == kNS) ? 0 : buf + 1;
             const float *As = stage + a_row * TL::RA + c_l;
             const float *Bs = stage + TL::A_WORDS + c_l * TL::PSB + b_col;
 #pragma unroll
@@ -312,8 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&empty_bar[buf]);  // this warp is done with the stage
         }
-
+        if (!ok) break;
         // Epilogue straight from registers.  A thread holds, per row m and k group q,
         // four consecutive k of its one l.  Shuffles among the lanes of a row group
         // turn that into four consecutive outputs of Y (DL >= 4: 4x4 transpose over
@@ -418,7 +429,6 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
             }
         }
     }
-    cp_async_wait<0>();  // no copy may still be landing when the CTA exits
 }
 
 template <int DL, int WM, int WK, int TN>
@@ -442,8 +452,10 @@ cudaError_t launch_cfg32(const Problem &pr, const float *vt) {
     const long long n_tiles = n_rb * p.n_g * p.n_kb;
     if (n_tiles > INT32_MAX - 4096) return cudaErrorInvalidConfiguration;  // tile indices are 32-bit
     p.n_tiles = (int)n_tiles;
-    const size_t smem = (size_t)TL::SMEM_FLOATS * sizeof(float);
+    const size_t smem = (size_t)((TL::SMEM_FLOATS * 4 + 15) / 16 * 16) + 2 * TL::NS * 8 + 16;
     if (smem > 232448) return cudaErrorInvalidConfiguration;
+    p.status = device_status_ptr();
+    if (!p.status) return cudaErrorUnknown;
     auto kern = vt ? fma32_kernel<DL, WM, WK, TN, true> : fma32_kernel<DL, WM, WK, TN, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

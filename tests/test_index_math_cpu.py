@@ -10,6 +10,8 @@ first GPU run; kept here so a change to the formulas must change them too.
 """
 import collections
 import math
+import os
+import re
 
 import pytest
 
@@ -108,6 +110,37 @@ def test_fma32_copies_cover_a_stage_once(tile):
     assert set(xs) == x_expect and set(xs.values()) == {1}
     assert set(vs) == v_expect and set(vs.values()) == {1}
     assert set(vts) == v_expect and set(vts.values()) == {1}
+
+
+def fma32_source():
+    path = os.path.join(os.path.dirname(__file__), "..", "kronecker_sparse_matrix_b200", "csrc", "ks_fma32.cu")
+    with open(path) as f:
+        return f.read()
+
+
+def test_fma32_copy_warpgroup_roles_barriers_and_register_split():
+    """The copy warpgroup's threads take each of a stage's 256 copy roles once,
+    the barrier counts match the arrivals, and the setmaxnreg split fits the
+    registers the block is launched with (a split above it would wait forever)."""
+    src = fma32_source()
+    threads = int(re.search(r"constexpr int kThreads = (\d+);", src).group(1))
+    roles = int(re.search(r"constexpr int kCopyRoles = (\d+);", src).group(1))
+    assert roles == THREADS and threads % 128 == 0
+    compute = 256  # warps 0-7 compute, warps 8.. issue copies
+    copy = threads - compute
+    # copy thread pt plays roles pt + copy * v, v < roles / copy
+    got = collections.Counter(pt + copy * v for pt in range(copy) for v in range(roles // copy))
+    assert roles % copy == 0 and set(got) == set(range(roles)) and set(got.values()) == {1}
+    # every copy thread makes one .noinc arrival per stage; every compute warp one arrival
+    full = int(re.search(r"mbar_init\(&full_bar\[s\], (\d+)\)", src).group(1))
+    empty = int(re.search(r"mbar_init\(&empty_bar\[s\], (\d+)\)", src).group(1))
+    assert full == copy and empty == compute // 32
+    dec = int(re.search(r"setmaxnreg\.dec\.sync\.aligned\.u32 (\d+)", src).group(1))
+    inc = int(re.search(r"setmaxnreg\.inc\.sync\.aligned\.u32 (\d+)", src).group(1))
+    # registers per thread at launch: 64K per SM over the launch bound, in units of 8
+    launch = (65536 // threads) // 8 * 8
+    assert dec % 8 == 0 and inc % 8 == 0 and 24 <= dec <= 256 and 24 <= inc <= 256
+    assert copy * dec + compute * inc <= threads * launch
 
 
 # ------------------------------------------------------------------ ks_tc.cu
