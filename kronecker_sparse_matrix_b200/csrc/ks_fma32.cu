@@ -35,6 +35,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "ks_epilogue.cuh"
 #include "ks_internal.h"
@@ -53,6 +54,7 @@ struct Fma32Params {
     const float *V;
     float *Y;
     const float *bias;  // fused epilogue: out_f values or null
+    int bias_vec4;      // bias is 16-byte aligned: read four columns at once
     int act;
     long long N;
     int a, b, c, d;
@@ -96,17 +98,16 @@ struct Tile32 {
     static constexpr int NXC = (BM * CA + kCopyRoles - 1) / kCopyRoles;  // A copies per role
 };
 
-// Fused bias and activation of four consecutive outputs (columns col..col+3).
-// Kept out of line: the epilogue is unrolled over every vector of a tile, and
-// inlining the activations there would bloat the kernel's code.
-__device__ __noinline__ float4 ep_vec4(float4 o, const float *bias, long long col, int act) {
-    float v[4] = {o.x, o.y, o.z, o.w};
-    if (bias) {
+// Activation ACT (0 none, 1 ReLU, 2 GELU tanh form, 3 GELU erf form) of four
+// outputs, chosen at compile time.
+template <int ACT>
+__device__ __forceinline__ void ep_act4(float (&v)[4]) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] += ep_bias(bias, col + e);
+    for (int e = 0; e < 4; ++e) {
+        if constexpr (ACT == 1) v[e] = fmaxf(v[e], 0.f);
+        if constexpr (ACT == 2) v[e] = gelu_tanh_f(v[e]);
+        if constexpr (ACT == 3) v[e] = gelu_erf_f(v[e]);
     }
-    if (act) ep_act_array(v, act);
-    return make_float4(v[0], v[1], v[2], v[3]);
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const float *src, bool valid) {
@@ -343,10 +344,12 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
         const int l_v = DL >= 4 ? l0 + (c_l & ~3) : l0;
         const int k_off = DL >= 4 ? r4 : DL == 2 ? 2 * c_l : 0;
         const long long colbase = (long long)i * p.b * p.d + l_v;
-        // Two copies of the unrolled store loop: the plain one carries no call
-        // site at all (the fused bias/activation's call, even when skipped, made
-        // the plain loop slower), the fused one calls the out-of-line helper.
-        if (p.bias == nullptr && p.act == 0) {
+        // The unrolled store loop, once per activation: the plain copy carries no
+        // epilogue code at all; the fused ones add the bias (read once per tile:
+        // the thread's TN/4 vectors of columns are the same for its 8 rows) and
+        // apply the activation inline.
+        auto store_tile = [&](auto act_c, const float4 *bq) {
+            constexpr int ACT = decltype(act_c)::value;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const long long row = n0 + a_row + LN::RG * m;
@@ -376,56 +379,41 @@ __global__ void __launch_bounds__(kThreads, 1) fma32_kernel(const Fma32Params p)
                         if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
                         else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
                     }
-                    const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
-                    if (row < p.N && k < p.b) {
-                        const long long off = (long long)k * p.d;
-                        float4 o = make_float4(v[0], v[1], v[2], v[3]);
-                        // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
-                        // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
-                        *reinterpret_cast<float4 *>(yrow + off) = o;
+                    if (bq) {
+                        v[0] += bq[q].x; v[1] += bq[q].y; v[2] += bq[q].z; v[3] += bq[q].w;
                     }
+                    ep_act4<ACT>(v);
+                    const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
+                    // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
+                    // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
+                    if (row < p.N && k < p.b)
+                        *reinterpret_cast<float4 *>(yrow + (long long)k * p.d) = make_float4(v[0], v[1], v[2], v[3]);
                 }
             }
+        };
+        if (p.bias == nullptr && p.act == 0) {
+            store_tile(std::integral_constant<int, 0>(), nullptr);
         } else {
+            float4 bq[TN / 4];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const long long row = n0 + a_row + LN::RG * m;
-                float *yrow = p.Y + row * p.out_f + colbase;
-#pragma unroll
-                for (int q = 0; q < TN / 4; ++q) {
-                    float v[4] = {acc[m][2 * q].x, acc[m][2 * q].y, acc[m][2 * q + 1].x, acc[m][2 * q + 1].y};
-                    if constexpr (DL >= 4) {
-                        // v[e] = (k + e, l = r4) over lanes r4 = 0..3  ->  v[e] = (k + r4, l = e)
-#pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const float snd = (r4 & 1) ? v[2 * t] : v[2 * t + 1];
-                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
-                            if (r4 & 1) v[2 * t] = rcv; else v[2 * t + 1] = rcv;
-                        }
-#pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const float snd = (r4 & 2) ? v[t] : v[t + 2];
-                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
-                            if (r4 & 2) v[t] = rcv; else v[t + 2] = rcv;
-                        }
-                    } else if constexpr (DL == 2) {
-                        // lanes l = 0, 1 (lane bit 1): l = 0 takes (k, k+1) x (l0, l1), l = 1 takes (k+2, k+3)
-                        const float s0 = c_l ? v[0] : v[2], s1 = c_l ? v[1] : v[3];
-                        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
-                        const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
-                        if (c_l) { v[0] = r0; v[1] = v[2]; v[2] = r1; }
-                        else { v[3] = r1; v[2] = v[1]; v[1] = r0; }
-                    }
-                    const int k = kt + 4 * LN::KQ * q + k_off;  // first k of the vector
-                    if (row < p.N && k < p.b) {
-                        const long long off = (long long)k * p.d;
-                        float4 o = make_float4(v[0], v[1], v[2], v[3]);
-                        // the vector's four outputs are consecutive columns of Y (DL >= 4: (k, l_v + e);
-                        // DL = 2 = d: (k + e/2, l0 + e%2); DL = 1: k + e)
-                        o = ep_vec4(o, p.bias, colbase + off, p.act);
-                        *reinterpret_cast<float4 *>(yrow + off) = o;
-                    }
+            for (int q = 0; q < TN / 4; ++q) {
+                const int k = kt + 4 * LN::KQ * q + k_off;
+                const long long col = colbase + (long long)k * p.d;
+                bq[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.bias && k < p.b) {
+                    if (p.bias_vec4)
+                        bq[q] = __ldg(reinterpret_cast<const float4 *>(p.bias + col));
+                    else
+                        bq[q] = make_float4(__ldg(p.bias + col), __ldg(p.bias + col + 1), __ldg(p.bias + col + 2),
+                                            __ldg(p.bias + col + 3));
                 }
+            }
+            const float4 *bp = p.bias ? bq : nullptr;
+            switch (p.act) {
+                case 1: store_tile(std::integral_constant<int, 1>(), bp); break;
+                case 2: store_tile(std::integral_constant<int, 2>(), bp); break;
+                case 3: store_tile(std::integral_constant<int, 3>(), bp); break;
+                default: store_tile(std::integral_constant<int, 0>(), bp); break;
             }
         }
     }
@@ -439,6 +427,7 @@ cudaError_t launch_cfg32(const Problem &pr, const float *vt) {
     p.V = vt ? vt : static_cast<const float *>(pr.V);
     p.Y = static_cast<float *>(pr.Y);
     p.bias = static_cast<const float *>(pr.bias);
+    p.bias_vec4 = (reinterpret_cast<uintptr_t>(pr.bias) % 16) == 0;
     p.act = pr.act;
     p.N = pr.batch;
     p.a = (int)pr.a; p.b = (int)pr.b; p.c = (int)pr.c; p.d = (int)pr.d;

@@ -11,8 +11,8 @@
 //     D_l[n, k] = sum_j A_l[n, j] * B_l[k, j],  A_l = X[:, i, :, l],  B_l = values[i, l]
 // with M = 128 rows of the batch, N = the k of one pass, K = c.
 //
-// A tile is 128 rows x one block i x DLS consecutive l (DLS = 8 when d % 8 ==
-// 0, else DLS = d).  Its outputs for all l and all k of a pass (DLS * bp <=
+// A tile is 128 rows x one block i x DLS consecutive l (DLS = 16 for bf16
+// when d % 16 == 0, DLS = 8 when d % 8 == 0, else DLS = d).  Its outputs for all l and all k of a pass (DLS * bp <=
 // 512 fp32 columns) accumulate in tensor memory while X streams through a
 // ring of 16/32 KB chunks exactly once per pass; most patterns need a single
 // pass, so X is read once and Y written once.  Each pass is its own tile, and
@@ -36,7 +36,9 @@
 //   warps 2..5  (DLS > 1) transpose each chunk in place, in registers, from
 //               [row][j][l] to one MN-major no-swizzle operand plane per l,
 //               padded (and, for bf16, skewed) so that every quarter-warp's
-//               16-byte accesses reach eight bank groups; for d = 1 the TMA box
+//               16-byte accesses reach eight bank groups (for DLS = 16 each
+//               warp transposes whole 8-row groups within their own 4 KB,
+//               unpadded); for d = 1 the TMA box
 //               already lands as the 128-byte-swizzled K-major tile the MMA
 //               reads, and these warps idle;
 //   warp 1      one thread issues tcgen05.mma (M=128, N=bp, K=32 bytes) per
@@ -45,7 +47,8 @@
 //               rows), convert to the storage type, interleave the l planes
 //               back into Y's (k, l) order in a shared-memory staging box of 32
 //               rows, and hand it to a TMA tensor store when the box is
-//               contiguous in Y (d == DLS); for fp32 with d > DLS, to a 4-D
+//               contiguous in Y (d == DLS); for 32-byte l runs (fp32
+//               with DLS = 8, bf16 with DLS = 16) and d > DLS, to a 4-D
 //               tensor store whose box is [k][row][l] (32-byte runs of Y);
 //               otherwise copy it out in 16-byte stores.
 //
@@ -84,12 +87,16 @@ constexpr int kLoadWarp0 = 2;      // warps 2..5
 constexpr int kEpiWarp0 = 6;       // warps 6..9
 constexpr int kEpiWarpBytes = 4096; // staging per epilogue warp: one box of 32 rows x 128 B
 constexpr int kChunkBytes = 128;    // output bytes per row per epilogue chunk
+constexpr int kBiasBytes = 2048;    // fused bias of one tile (bp * DLS * ES <= 2 KB), per buffer and warp
 constexpr int kSmemLimit = 232448; // per-block opt-in maximum on sm_100
 
 // j per MMA (K = 32 bytes): 16 bf16, 8 fp32 (TF32)
 __host__ __device__ constexpr int step_j(int es) { return 32 / es; }
-// j per X chunk: raw rows of 256 bytes for DLS = 8, 128 bytes otherwise
-__host__ __device__ constexpr int chunk_j(int dls, int es) { return (dls == 8 ? 32 : 128 / dls) / es; }
+// j per X chunk: raw rows of 256 bytes for DLS = 8, 128 bytes for DLS < 8;
+// DLS = 16 (bf16 only) takes one K step, 16 j x 16 l = 512-byte rows
+__host__ __device__ constexpr int chunk_j(int dls, int es) {
+    return dls == 16 ? 16 : (dls == 8 ? 32 : 128 / dls) / es;
+}
 __host__ __device__ constexpr int chunk_bytes(int dls, int es) { return kRows * chunk_j(dls, es) * dls * es; }
 // Transposed operand planes (DLS > 1), one per l.
 //   bf16: MN-major, no swizzle: core matrices of 8 j lines x 16 bytes (8
@@ -101,6 +108,11 @@ __host__ __device__ constexpr int chunk_bytes(int dls, int es) { return kRows * 
 //         K step) per batch row, 128 rows = 4 KB per j octet (the tensor
 //         cores read TF32 operands K-major; the layout is the one the values
 //         operand uses for rows of 32 bytes).
+//   bf16 with DLS = 16: the planes of the 8 rows of a row group take the
+//         4 KB the group's raw rows took (core matrix (l, j octet) at
+//         (2 l + octet) * 128 bytes), so each group is transposed in place by
+//         one warp, without padding: its lanes' units are chosen so that
+//         every quarter-warp reaches eight bank groups in both directions.
 __host__ __device__ constexpr int group_stride(int es) { return es == 2 ? 144 : 256; }
 __host__ __device__ constexpr int octet_stride(int es) { return es == 2 ? 16 * 144 : 128 * 32; }
 __host__ __device__ constexpr int plane_stride(int dls, int es) { return (chunk_j(dls, es) / 8) * octet_stride(es); }
@@ -109,8 +121,10 @@ __host__ __device__ constexpr int plane_stride(int dls, int es) { return (chunk_
 // after the X ring keep the 1 KiB alignment of the ring's base (the largest
 // swizzle atom: 8 rows x 128 bytes)
 __host__ __device__ constexpr int slot_bytes(int dls, int es) {
-    return (dls == 1 ? chunk_bytes(1, es) : dls * plane_stride(dls, es) + 1023) / 1024 * 1024;
+    return (dls == 1 || dls == 16 ? chunk_bytes(dls, es) : dls * plane_stride(dls, es) + 1023) / 1024 * 1024;
 }
+// DLS = 16 planes: bytes between row groups (8 raw rows of 512 bytes)
+constexpr int kG16 = 4096;
 // The values of one chunk land as DLS planes of bp rows (k) x chunk_j j,
 // K-major with the swizzle as wide as a row (chunk_j * es bytes): tcgen05
 // layout type and the TMA swizzle mode for that width.
@@ -137,7 +151,7 @@ struct TcParams {
     int box_elems, box_sw128;        // epilogue staging box: elements per row, swizzled
     int box_row_bytes;               // staging row stride when not swizzled (an odd number of 16-byte units)
     int ytma;                        // the staging box goes to Y as one TMA store: 2-D (d == DLS) or,
-                                     // in the Y4 kernels, 4-D ([k][row][l] box, fp32 with d > DLS)
+                                     // in the Y4 kernels, 4-D ([k][row][l] box, DLS * ES = 32, d > DLS)
     int x3d;                         // X chunks come from the (c*d, a, N) map (DLS < 8, or d == 8)
 };
 
@@ -151,6 +165,14 @@ __device__ __forceinline__ void mma_kind(uint32_t d_tmem, uint64_t adesc, uint64
         mma_tf32(d_tmem, adesc, bdesc, idesc, accumulate);
 }
 
+// 16-byte global -> shared copy (L2 only), its commit and the wait for all of
+// this thread's copies.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // 4x4 transpose of 32-bit elements: in[r] holds elements e=0..3 of row r;
 // out[e] holds rows r=0..3 of element e (a renaming of registers).
 __device__ __forceinline__ void transpose4x4_b32(const uint4 (&in)[4], uint4 (&out)[4]) {
@@ -161,7 +183,7 @@ __device__ __forceinline__ void transpose4x4_b32(const uint4 (&in)[4], uint4 (&o
 }
 
 // EP: fused bias / activation epilogue compiled in; Y4: the output boxes go to
-// a 4-D TMA store of [k][row][l] boxes (fp32 with d > DLS), chosen at compile
+// a 4-D TMA store of [k][row][l] boxes (32-byte l runs, d > DLS), chosen at compile
 // time so that the other instantiations carry none of it (a run-time choice
 // cost the d == DLS TF32 epilogue 5-7%).
 template <int DLS, typename T, bool EP, bool Y4 = false>
@@ -243,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = mbar_wait(&x_empty[xs], ((xq / S) & 1) ^ 1, abort_flag, p.status, wait_ns);
                     if (!ok) break;
                     mbar_expect_tx(&x_full[xs], (uint32_t)CB);
-                    if (DLS == 8 && !p.x3d)
+                    if (DLS >= 8 && !p.x3d)
                         tma_load_4d(sR + xs * SB, &xmap, &x_full[xs], l0, ch * CTJ, i, n0);
                     else
                         tma_load_3d(sR + xs * SB, &xmap, &x_full[xs], ch * CTJ * p.d, i, n0);
@@ -305,6 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint64_t ad;
                             if (DLS == 1)
                                 ad = smem_desc_sw128(stage + sl * 32, 1024);
+                            else if (DLS == 16)  // MN-major, group-local planes: one K step per chunk
+                                ad = smem_desc(stage + l * 256, 128, kG16);
                             else if (ES == 2)  // MN-major: a K step spans two j octets of the plane
                                 ad = smem_desc(stage + l * PS + sl * 2 * OS, OS, GS);
                             else  // K-major, 32-byte swizzle: a K step is one j octet, 8-row atoms 256 bytes apart
@@ -326,7 +350,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------ in-place transpose (DLS > 1)
-        if (DLS > 1 && ES == 2) {
+        if constexpr (DLS == 16) {
+            // bf16, 16 l: raw row = 32 units of 16 bytes, unit q = (j = q / 2,
+            // l half q % 2).  Warp tw takes row groups tw, tw + 4, tw + 8, tw + 12;
+            // per group each lane reads one unit of the 8 rows, transposes it
+            // and, after the whole warp has read, writes 8 lines (row group g,
+            // l = 8 h + e, j) of the planes into the same 4 KB.  Lanes of a
+            // quarter-warp take j = 0..7 (+8) with the l half flipped for the
+            // upper four, so their reads (bank group q % 8) and their writes
+            // (bank group j % 8) reach eight bank groups each.
+            const int tw = warp - kLoadWarp0;  // 0..3
+            const int quarter = lane >> 3, idx = lane & 7;
+            const int h = (idx >> 2) ^ (quarter & 1);
+            const int j = 8 * (quarter >> 1) + idx;
+            const int q = 2 * j + h;
+            uint32_t xq = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+                for (int ch = 0; ch < n_chunks; ++ch, ++xq) {
+                    const int xs = xq % S;
+                    const bool w = mbar_wait(&x_full[xs], (xq / S) & 1, abort_flag, p.status, wait_ns);
+                    ok = bar_and(1, 128, w);  // uniform over the four loader warps
+                    if (!ok) break;
+                    uint8_t *st = sR + xs * SB;
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        uint8_t *gb = st + (4 * it + tw) * kG16;
+                        uint4 in[8], out[8];
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) in[r] = *reinterpret_cast<const uint4 *>(gb + r * 512 + q * 16);
+                        transpose8x8_b16(in, out);
+                        __syncwarp();  // every lane has read the group
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            *reinterpret_cast<uint4 *>(gb + (2 * (8 * h + e) + (j >> 3)) * 128 + (j & 7) * 16) = out[e];
+                    }
+                    fence_proxy_async();
+                    mbar_arrive(&a_ready[xs]);
+                }
+            }
+        } else if (DLS > 1 && ES == 2) {
             const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
             // task -> (16-byte unit q of a raw row, group g of 8 rows).  16-byte
             // shared accesses are served eight lanes at a time, so every eight
@@ -471,6 +534,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         // staging row stride (not sw): dense rows for the tensor store, else padded rows
         const int rsb = p.ytma ? p.box_elems * ES : p.box_row_bytes;
         const T *bias = static_cast<const T *>(p.bias);
+        // Fused bias, DLS >= 4: the tile's bp x DLS columns, 16-byte units in
+        // (k, l) order, go with cp.async to one of two buffers of this warp while
+        // the warp drains the previous tile, so no chunk waits for a global load
+        // (and no warp waits for another).  With DLS <= 2 a chunk's bias is one
+        // contiguous 128-byte line that the chunk reads from L1 directly, which
+        // measured faster there (d = 1, 2: 0.86-0.95x with the copies).
+        constexpr bool kBiasSmem = DLS >= 4;
+        uint8_t *sB = sE + 4 * kEpiWarpBytes + ew * 2 * kBiasBytes;
+        auto bias_prefetch = [&](long long tile, int slot) {
+            const int ps = (int)(tile % p.passes);
+            const int g = (int)((tile / p.passes) % p.n_g);
+            const int i = g / groups_per_i, l0 = (g % groups_per_i) * DLS;
+            const int nu = p.bp * DLS / RPU;  // at most 128
+            for (int U = lane; U < nu; U += 32) {
+                const int f = RPU * U;  // first (k, l) element of the unit
+                const T *src = bias + (long long)i * p.b * p.d + l0 + (long long)(ps * p.bp + f / DLS) * p.d + f % DLS;
+                cp_async16(su32(sB) + slot * kBiasBytes + U * 16, src);
+            }
+            cp_async_commit();
+        };
+        if (EP && kBiasSmem && bias && blockIdx.x < p.n_tiles) bias_prefetch(blockIdx.x, 0);
         uint32_t accq = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++accq) {
@@ -483,7 +567,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int buf = (int)(accq % p.nbuf);
             ok = mbar_wait(&acc_full[buf], (accq / p.nbuf) & 1, abort_flag, p.status, wait_ns);
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+            if (EP && kBiasSmem && bias) {
+                // this tile's bias has landed (every lane's copies, shown to the warp
+                // by the sync); the other buffer, last read for the previous tile,
+                // takes the next tile's
+                cp_async_wait_all();
+                __syncwarp();
+                if (ok && tile + gridDim.x < p.n_tiles) bias_prefetch(tile + gridDim.x, (accq + 1) & 1);
+            }
             if (!ok) break;
+            const uint8_t *bias_tile = sB + (accq & 1) * kBiasBytes;
             tc_fence_after();
             for (int oc = 0; oc < n_oc; ++oc) {
                 float acc[DLS][KCM];
@@ -516,14 +609,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kq = ps * p.bp + oc * kc;  // first k of the chunk
                 const long long ybase = (long long)i * p.b * p.d + l0;
                 if (EP && bias) {
-                    // fused epilogue on (k = kq + e, l): the chunk's bias in 16-byte units of
-                    // RPU consecutive l of one k (the same for every lane: one transaction each)
+                    // fused epilogue on (k = kq + e, l): the chunk's bias, units oc * units + u
+                    // of the tile's copy, or 16-byte units of RPU consecutive (k, l) read
+                    // directly (either way the same address for every lane: a broadcast)
 #pragma unroll
                     for (int u = 0; u < CE / RPU; ++u) {
                         if (u < units) {
-                            const int e0 = (RPU * u) / DLS, lu = (RPU * u) % DLS;
-                            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(bias + ybase +
-                                                                                  (long long)(kq + e0) * p.d + lu));
+                            uint4 w;
+                            if constexpr (kBiasSmem) {
+                                w = *reinterpret_cast<const uint4 *>(bias_tile + (oc * units + u) * 16);
+                            } else {
+                                const int e0 = (RPU * u) / DLS, lu = (RPU * u) % DLS;
+                                w = __ldg(reinterpret_cast<const uint4 *>(bias + ybase + (long long)(kq + e0) * p.d + lu));
+                            }
                             float bb[RPU];
                             if constexpr (ES == 2) {
                                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
@@ -571,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         uint32_t off = sw ? lane * 128 + ((u ^ (lane & 7)) << 4) : lane * rsb + u * 16;
-                        // 4-D box (fp32 only): [k][row][l], unit u = (k, l0u .. l0u + RPU - 1); the
+                        // 4-D box (DLS * ES = 32): [k][row][l], unit u = (k, l0u .. l0u + RPU - 1); the
                         // eight lanes of a 16-byte store reach at least four bank groups
                         if constexpr (Y4)
                             off = ((RPU * u) / DLS) * (32 * DLS * ES) + lane * (DLS * ES) + ((RPU * u) % DLS) * ES;
@@ -644,7 +742,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// bf16 takes 16 l per tile where that measured faster than 8 on all 66 bf16
+// sweep patterns with d >= 16 at 25088 rows: d a multiple of 64 with c <= 96
+// (X boxes of 32-byte rows instead of 16; 1.05-1.17x), and d = 16 with b not a
+// multiple of 32 (passes of 16 k with double-buffered accumulators; 1.02-1.15x).
+// Elsewhere the passes of at most 32 k, which repeat the copy and transpose of
+// every X chunk twice as often as 8 l with 64 k, made it 0.77-0.99x.
 int tc_dls(const Problem &p) {
+    if (p.dtype == KS_BF16 && p.d % 16 == 0 && ((p.d % 64 == 0 && p.c <= 96) || (p.d == 16 && p.b % 32 != 0)))
+        return 16;
     if (p.d % 8 == 0) return 8;
     if (p.d == 1 || p.d == 2 || p.d == 4) return (int)p.d;
     return 0;
@@ -683,17 +789,29 @@ constexpr int kBarBytes = (3 * kMaxStages + 2 * kVStages + 2 + 2 + 1) * 8 + 16;
 
 // Shared memory: the X ring (as deep as fits, 3..8 chunks), the values ring
 // (one stage per X chunk: DLS planes x bp k x CTJ j, 3..4 deep), the epilogue
-// staging, barriers.
-bool tc_layout(int dls, int bp, int es, TcLayout *out) {
+// staging (and, with a fused bias and DLS >= 4, two tiles of bias per epilogue
+// warp), barriers.
+bool tc_layout(int dls, int bp, int es, bool bias, TcLayout *out) {
+    const bool ep = bias && dls >= 4;
     TcLayout L;
     auto up = [](int x, int a) { return (x + a - 1) / a * a; };
     const int cb = slot_bytes(dls, es);
     L.v_stage_bytes = es * bp * chunk_j(dls, es) * dls;
-    const int epi = 4 * kEpiWarpBytes;
-    const int budget = kSmemLimit - 2048 - epi - kBarBytes;  // alignment slack
+    if (bp * dls * es > kBiasBytes) return false;
+    const int epi = 4 * kEpiWarpBytes + (ep ? 4 * 2 * kBiasBytes : 0);
+    const int budget = kSmemLimit - 2048 - 4 * kEpiWarpBytes - kBarBytes;  // alignment slack
+    auto x_stages = [&](int bud, int vs) {
+        return std::min(kMaxStages, (bud - up(vs * L.v_stage_bytes, 128)) / cb);
+    };
     L.vstages = (kVStages * L.v_stage_bytes + 3 * cb <= budget) ? kVStages : 3;
-    const int left = budget - up(L.vstages * L.v_stage_bytes, 128);
-    L.stages = std::min(kMaxStages, left / cb);
+    L.stages = x_stages(budget, L.vstages);
+    if (ep) {  // the bias buffers come out of a values stage rather than an X stage where possible
+        const int bud = budget - 4 * 2 * kBiasBytes;
+        int vs = L.vstages, st = x_stages(bud, vs);
+        if (st < L.stages && vs == kVStages && x_stages(bud, 3) > st) st = x_stages(bud, vs = 3);
+        L.vstages = vs;
+        L.stages = st;
+    }
     if (L.stages < 2) return false;
     L.off_v = L.stages * cb;
     L.off_epi = up(L.off_v + L.vstages * L.v_stage_bytes, 1024);
@@ -739,7 +857,7 @@ bool tc_supported(const Problem &p, const char **why) {
     const int bp = tc_bp(dls, p.b);
     TcLayout L;
     if (bp == 0 || tc_kc(dls, bp, es) == 0) { *why = "b has no pass width (a multiple of 16 dividing it)"; return false; }
-    if (!tc_layout(dls, bp, es, &L)) { *why = "shared memory budget"; return false; }
+    if (!tc_layout(dls, bp, es, p.bias != nullptr, &L)) { *why = "shared memory budget"; return false; }
     if (p.batch > (1LL << 31) - 256 || p.a * p.d > (1LL << 31)) { *why = "sizes exceed tensor-map coordinates"; return false; }
     return true;
 }
@@ -752,22 +870,22 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     if (!encode) return cudaErrorNotSupported;
     const int bp = cfg.bk;
     TcLayout L;
-    if (bp == 0 || !tc_layout(DLS, bp, ES, &L)) return cudaErrorInvalidConfiguration;
+    if (bp == 0 || !tc_layout(DLS, bp, ES, pr.bias != nullptr, &L)) return cudaErrorInvalidConfiguration;
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap xmap, vmap;
     CUresult r;
-    const bool x3d = DLS < 8 || pr.d == 8;
+    const bool x3d = DLS < 8 || pr.d == DLS;
     if (!x3d) {
-        // X as (d, c, a, N): a box (8 l, CTJ j, 1, 128 rows) = [row][j][l]
+        // X as (d, c, a, N): a box (DLS l, CTJ j, 1, 128 rows) = [row][j][l]
         cuuint64_t dims[4] = {(cuuint64_t)pr.d, (cuuint64_t)pr.c, (cuuint64_t)pr.a, (cuuint64_t)pr.batch};
         cuuint64_t strides[3] = {(cuuint64_t)pr.d * ES, (cuuint64_t)pr.c * pr.d * ES,
                                  (cuuint64_t)pr.in_features() * ES};
-        cuuint32_t box[4] = {8, (cuuint32_t)chunk_j(8, ES), 1, (cuuint32_t)kRows};
+        cuuint32_t box[4] = {(cuuint32_t)DLS, (cuuint32_t)chunk_j(DLS, ES), 1, (cuuint32_t)kRows};
         r = encode(&xmap, kType, 4, const_cast<void *>(pr.X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
         // X as (c*d, a, N): a box (CTJ*DLS elements, 1, 128 rows) = [row][(j, l)]
-        // (d == DLS, or d == 8: whole 256-byte rows); for d == 1 with the
+        // (d == DLS: whole 256- or 512-byte rows for DLS = 8 or 16); for d == 1 with the
         // 128-byte swizzle, the K-major operand tile itself
         cuuint64_t dims[3] = {(cuuint64_t)(pr.c * pr.d), (cuuint64_t)pr.a, (cuuint64_t)pr.batch};
         cuuint64_t strides[2] = {(cuuint64_t)pr.c * pr.d * ES, (cuuint64_t)pr.in_features() * ES};
@@ -801,11 +919,13 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     const bool sw128 = bi * ES == kChunkBytes;
     const bool yal = (reinterpret_cast<uintptr_t>(pr.Y) % 16) == 0;
     const bool ytma = pr.d == DLS && yal;
-    // fp32 with d > DLS: Y viewed as (d, N, b, a), a box (DLS l, 32 rows, kc k,
-    // 1 block) whose shared image is [k][row][l] with 32-byte (k, row) runs and
-    // no swizzle.  (Measured against the 16-byte stores: 1.11x median on the
-    // d >= 16 TF32 patterns; for bf16 the 16-byte runs made it slower.)
-    const bool y4d = ES == 4 && DLS == 8 && pr.d > DLS && yal;
+    // 32-byte l runs (fp32 with DLS = 8, bf16 with DLS = 16) and d > DLS: Y
+    // viewed as (d, N, b, a), a box (DLS l, 32 rows, kc k, 1 block) whose
+    // shared image is [k][row][l] with 32-byte (k, row) runs and no swizzle.
+    // (Measured against the 16-byte stores: 1.11x median on the d >= 16 TF32
+    // patterns; for bf16 with DLS = 8 the 16-byte runs made it slower.)
+    constexpr bool kY4 = DLS * ES == 32;
+    const bool y4d = kY4 && pr.d > DLS && yal;
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
     if (y4d) {
@@ -861,7 +981,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.v_stage_bytes = L.v_stage_bytes;
     const bool ep = pr.bias || pr.act;
     auto kern = ep ? tc_kernel<DLS, T, true> : tc_kernel<DLS, T, false>;
-    if constexpr (ES == 4 && DLS == 8)
+    if constexpr (kY4)
         if (y4d) kern = ep ? tc_kernel<DLS, T, true, true> : tc_kernel<DLS, T, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (e != cudaSuccess) return e;
@@ -873,6 +993,9 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
 template <typename T>
 static cudaError_t launch_typed(const Problem &p, const TcConfig &cfg) {
     switch (cfg.dl) {
+        case 16:
+            if constexpr (sizeof(T) == 2) return launch_dls<16, T>(p, cfg);
+            return cudaErrorInvalidConfiguration;
         case 8: return launch_dls<8, T>(p, cfg);
         case 4: return launch_dls<4, T>(p, cfg);
         case 2: return launch_dls<2, T>(p, cfg);

@@ -24,7 +24,8 @@ CASES = [((2, 4, 4, 2), torch.float32, "stream"), ((4, 2, 2, 1), torch.float32, 
          ((1, 48, 48, 8), torch.bfloat16, "fma"),
          ((1, 192, 48, 8), torch.bfloat16, "tc"), ((2, 64, 64, 1), torch.bfloat16, "tc"),
          ((1, 64, 64, 2), torch.bfloat16, "tc"), ((1, 128, 64, 4), torch.bfloat16, "tc"),
-         ((1, 256, 64, 16), torch.bfloat16, "tc")]
+         ((1, 256, 64, 16), torch.bfloat16, "tc"), ((2, 64, 32, 64), torch.bfloat16, "tc"),
+         ((1, 48, 48, 16), torch.bfloat16, "tc")]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[0]}-{str(c[1])[6:]}-{c[2]}")

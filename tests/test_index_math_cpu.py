@@ -146,7 +146,16 @@ def test_fma32_copy_warpgroup_roles_barriers_and_register_split():
 # ------------------------------------------------------------------ ks_tc.cu
 # es = element bytes: 2 (bf16, kind::f16) or 4 (fp32 read as TF32, kind::tf32).
 def chunk_j(dls, es=2):
-    return (32 if dls == 8 else 128 // dls) // es
+    return 16 if dls == 16 else (32 if dls == 8 else 128 // dls) // es
+
+
+def tc_dls(p, es):
+    """l per tile: 16 for bf16 with d % 64 == 0 and c <= 96, or d = 16 and b %
+    32 != 0; 8 for d % 8 == 0; else d."""
+    a, b, c, d = p
+    if es == 2 and d % 16 == 0 and ((d % 64 == 0 and c <= 96) or (d == 16 and b % 32)):
+        return 16
+    return 8 if d % 8 == 0 else d
 
 
 def group_stride(es):
@@ -163,7 +172,7 @@ def plane_stride(dls, es):
 
 def slot_bytes(dls, es):
     raw = 128 * chunk_j(dls, es) * dls * es
-    return (raw if dls == 1 else dls * plane_stride(dls, es) + 1023) // 1024 * 1024
+    return (raw if dls in (1, 16) else dls * plane_stride(dls, es) + 1023) // 1024 * 1024
 
 
 def tc_task_unit(dls, task, units):
@@ -238,6 +247,73 @@ def test_tc_bf16_mma_descriptor_reads_what_the_transposer_wrote(dls):
                 for k in range(16):
                     addr = start + (m // 8) * gs + (k // 8) * os_ + (k % 8) * 16 + (m % 8) * es
                     assert addr == where[(m, 16 * s + k, l)]
+
+
+def dls16_transposer():
+    """bf16 with 16 l: warp tw, group g = 4 it + tw; lane -> raw unit q =
+    (j, l half h); reads rows r of unit q, writes line (l = 8 h + e, j) of the
+    group's planes.  Returns per group the lanes' (read addresses per r,
+    write addresses per e, j, h), addresses relative to the slot."""
+    g16 = 4096
+    out = {}
+    for tw in range(4):
+        for it in range(4):
+            g = 4 * it + tw
+            lanes = []
+            for lane in range(32):
+                quarter, idx = lane >> 3, lane & 7
+                h = (idx >> 2) ^ (quarter & 1)
+                j = 8 * (quarter >> 1) + idx
+                q = 2 * j + h
+                reads = [g * g16 + r * 512 + q * 16 for r in range(8)]
+                writes = [g * g16 + (2 * (8 * h + e) + (j >> 3)) * 128 + (j & 7) * 16 for e in range(8)]
+                lanes.append((reads, writes, j, h, q))
+            out[g] = lanes
+    return out
+
+
+def test_tc_bf16_dls16_transposer_is_in_place_and_conflict_free():
+    """Each warp's group: the lanes' units cover the 8 rows' 4 KB once, the
+    writes land inside the same 4 KB, once each, and every quarter-warp's
+    16-byte reads and writes reach eight distinct bank groups."""
+    slot = slot_bytes(16, 2)
+    assert slot == 128 * 512 == 128 * chunk_j(16, 2) * 16 * 2
+    tr = dls16_transposer()
+    assert sorted(tr) == list(range(16))
+    for g, lanes in tr.items():
+        assert sorted(q for *_, q in lanes) == list(range(32))
+        lo, hi = g * 4096, g * 4096 + 4096
+        reads = [a for rd, *_ in lanes for a in rd]
+        writes = [a for _, wr, *_ in lanes for a in wr]
+        assert sorted(reads) == list(range(lo, hi, 16)) and sorted(writes) == list(range(lo, hi, 16))
+        for q0 in range(0, 32, 8):
+            quarter = lanes[q0:q0 + 8]
+            for r in range(8):
+                assert len({(rd[r] // 16) % 8 for rd, *_ in quarter}) == 8
+            for e in range(8):
+                assert len({(wr[e] // 16) % 8 for _, wr, *_ in quarter}) == 8
+
+
+def test_tc_bf16_dls16_mma_descriptor_reads_what_the_transposer_wrote():
+    """Plane l's A operand for the chunk's one K step: MN-major no swizzle,
+    element (row m, k) at l * 256 + (m // 8) * SBO + (k // 8) * LBO + (k % 8) *
+    16 + (m % 8) * 2 with LBO = 128, SBO = 4096; it must hold X[row m][j = k][l]."""
+    where = {}
+    for g, lanes in dls16_transposer().items():
+        for reads, writes, j, h, q in lanes:
+            for e in range(8):
+                for r in range(8):  # line e holds element e of unit q for rows 0..7
+                    where[(8 * g + r, j, 8 * h + e)] = writes[e] + 2 * r
+    assert len(where) == 128 * 16 * 16 and len(set(where.values())) == len(where)
+    for l in range(16):
+        for m in range(128):
+            for k in range(16):
+                addr = l * 256 + (m // 8) * 4096 + (k // 8) * 128 + (k % 8) * 16 + (m % 8) * 2
+                assert addr == where[(m, k, l)]
+    # the raw row is [j][l], 16 l per j: unit q = 2 j + h holds l = 8 h .. 8 h + 7
+    for g, lanes in dls16_transposer().items():
+        for reads, writes, j, h, q in lanes:
+            assert q * 16 == (j * 16 + 8 * h) * 2
 
 
 def tf32_tasks(dls):
@@ -367,14 +443,15 @@ def tc_kc(dls, bp, es=2):
 @pytest.mark.parametrize("es", [2, 4])
 @pytest.mark.parametrize("p", [(2, 48, 48, 2), (1, 48, 48, 4), (2, 64, 64, 16), (1, 192, 48, 8), (3, 32, 16, 4),
                                (1, 256, 256, 2), (2, 48, 48, 1), (1, 16, 16, 1), (1, 96, 96, 4), (1, 80, 16, 2),
-                               (1, 48, 8, 1), (2, 256, 64, 16)])
+                               (1, 48, 8, 1), (2, 256, 64, 16), (1, 48, 48, 32), (2, 96, 64, 64), (1, 48, 32, 16),
+                               (1, 48, 48, 64), (1, 192, 48, 64)])
 def test_tc_epilogue_writes_each_output_once(p, es):
     """The output boxes of a tile: 32 rows x (DLS * kc) elements per warp and
     chunk, either one tensor store of a contiguous box (d == DLS), one 4-D
-    tensor store of a [k][row][l] box (fp32, d > DLS) or 16-byte stores of its
+    tensor store of a [k][row][l] box (32-byte l runs, d > DLS) or 16-byte stores of its
     units; N = 300 leaves a ragged last row block."""
     a, b, c, d = p
-    dls = 8 if d % 8 == 0 else d
+    dls = tc_dls(p, es)
     bp = tc_bp(dls, b)
     kc = tc_kc(dls, bp, es)
     assert kc > 0 and bp % kc == 0 and dls * kc * es <= 128
@@ -400,7 +477,7 @@ def test_tc_epilogue_writes_each_output_once(p, es):
                                 for r in range(min(32, n - row0)):
                                     for e in range(dls * kc):
                                         written[(row0 + r, x + e)] += 1
-                            elif es == 4:  # one 4-D box [k][row][l] of Y viewed as (d, N, b, a)
+                            elif dls * es == 32:  # one 4-D box [k][row][l] of Y viewed as (d, N, b, a)
                                 if row0 >= n:
                                     continue
                                 assert (l0 * es) % 16 == 0 and kq + kc <= b
@@ -421,8 +498,7 @@ def test_tc_epilogue_writes_each_output_once(p, es):
     assert len(written) == n * out_f and set(written.values()) == {1}
 
 
-@pytest.mark.parametrize("es", [2, 4])
-@pytest.mark.parametrize("dls", [1, 2, 4, 8])
+@pytest.mark.parametrize("dls,es", [(1, 2), (2, 2), (4, 2), (8, 2), (16, 2), (1, 4), (2, 4), (4, 4), (8, 4)])
 def test_tc_shared_memory_offsets_keep_their_alignment(dls, es):
     """Every X ring slot is a TMA destination (128-byte aligned at least, 1 KiB
     for the 128-byte swizzle of d = 1), and the values ring that follows the X
@@ -445,15 +521,15 @@ def test_tc_shared_memory_offsets_keep_their_alignment(dls, es):
                     assert (off_v + vs * vstage + l * plane) % atom == 0
 
 
-@pytest.mark.parametrize("es", [2, 4])
-def test_tc_4d_store_staging_is_the_box_in_order(es):
-    """fp32 with d > DLS: the epilogue writes unit u of row `lane` at
+@pytest.mark.parametrize("dls,es", [(8, 4), (16, 2), (8, 2)])
+def test_tc_4d_store_staging_is_the_box_in_order(dls, es):
+    """32-byte l runs (fp32 with DLS = 8, bf16 with DLS = 16) and d > DLS: the epilogue writes unit u of row `lane` at
     ((RPU u) / DLS) * 32 DLS es + lane * DLS es + ((RPU u) % DLS) es, which must
     be exactly the box (DLS l, 32 rows, kc k) in its shared order (l fastest,
     then row, then k), every byte once, within the 4 KB staging; eight lanes of
     one 16-byte store reach at least four bank groups.  (The bf16 form of this
-    layout is modelled too although bf16 keeps its 16-byte stores.)"""
-    dls, rpu = 8, 16 // es
+    layout with DLS = 8 is modelled too although it keeps 16-byte stores.)"""
+    rpu = 16 // es
     kc = (128 // es) // dls
     units = dls * kc * es // 16
     seen = set()
@@ -479,7 +555,9 @@ def test_tc_fused_bias_units_are_aligned_and_cover_the_chunk(es):
     """The tensor-core epilogue reads a chunk's bias as 16-byte units of RPU
     consecutive (k, l) outputs at bias + ybase + (kq + e0) * d + lu: every unit
     is 16-byte aligned (for a 16-byte-aligned bias) and the units cover the
-    chunk's kc x DLS columns exactly once, on sweep and test patterns."""
+    chunk's kc x DLS columns exactly once, on sweep and test patterns; the
+    tile's copy of them in shared memory puts each at the index the chunks
+    read."""
     from kronecker_sparse_matrix_b200 import inputs
     pats = inputs.sweep_patterns()[::5] + [(1, 192, 48, 8), (1, 256, 64, 16), (2, 64, 64, 2), (4, 64, 32, 1),
                                            (2, 48, 24, 2), (1, 32, 40, 4), (1, 16, 56, 8), (3, 32, 16, 4),
@@ -488,7 +566,7 @@ def test_tc_fused_bias_units_are_aligned_and_cover_the_chunk(es):
     for (a, b, c, d) in pats:
         if c % (32 // es):
             continue
-        dls = 8 if d % 8 == 0 else d
+        dls = tc_dls((a, b, c, d), es)
         bp = tc_bp(dls, b)
         kc = tc_kc(dls, bp, es) if bp else 0
         if not kc:
@@ -507,3 +585,18 @@ def test_tc_fused_bias_units_are_aligned_and_cover_the_chunk(es):
                         assert all(off + h == ybase + (kq + (rpu * u + h) // dls) * d + (rpu * u + h) % dls
                                    for h in range(rpu))
                     assert sorted(cols) == sorted(ybase + (kq + e) * d + l for e in range(kc) for l in range(dls))
+            # the tile's copy into shared memory: thread et < bp * DLS / RPU takes
+            # unit et = (k, l) element RPU * et of the tile, which is unit u of
+            # chunk oc for et = oc * units + u, and stays inside the bias
+            nu = bp * dls // rpu
+            assert nu <= 128 and nu * 16 <= 2048
+            for ps in range(b // bp):
+                ybase = i * b * d
+                for l0 in range(0, d, dls):
+                    for et in range(nu):
+                        f = rpu * et
+                        off = ybase + l0 + (ps * bp + f // dls) * d + f % dls
+                        oc, u = divmod(et, units)
+                        e0, lu = (rpu * u) // dls, (rpu * u) % dls
+                        assert off == ybase + l0 + (ps * bp + oc * kc + e0) * d + lu
+                        assert (off * es) % 16 == 0 and off + rpu <= a * b * d

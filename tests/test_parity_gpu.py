@@ -181,9 +181,12 @@ def test_full_size_sweep_patterns_sampled_rows(idx, dtype):
 # Full-size sweep patterns compared on every row: the tensor-core kernel's l
 # widths 1 (48 and 256 x 64 blocks, a = 64 and 8), 2, 4, 8 with d = 8 (whole
 # 256-byte rows) and 8 with d >= 16 (four-dimensional boxes), the last with
-# several k passes per X tile (b = 96, 128 with d = 16, 32); the fp32 kernel's
-# l widths 1, 2, 4, 8 (d >= 16 with the transposed-values workspace).
-FULL_ROWS = [82, 205, 127, 48, 248, 117, 36, 234]
+# several k passes per X tile (b = 96, 128 with d = 16, 32); in bf16, 16 l with
+# d = 16 and b = 48 (whole 512-byte rows, passes of 16 k, contiguous output
+# boxes) and with d = 64 (four-dimensional boxes both ways, six passes); the
+# fp32 kernel's l widths 1, 2, 4, 8 (d >= 16 with the transposed-values
+# workspace).
+FULL_ROWS = [82, 205, 127, 48, 248, 117, 36, 234, 4, 208]
 
 
 @pytest.mark.parametrize("idx", FULL_ROWS)
@@ -198,7 +201,9 @@ def test_full_size_sweep_patterns_every_row(idx, dtype):
 
 
 TC_CASES = [(1, 64, 64, 1), (1, 48, 48, 1), (2, 64, 64, 2), (1, 256, 64, 16), (1, 96, 96, 4), (4, 128, 128, 1),
-            (1, 48, 48, 8), (2, 192, 48, 8), (1, 256, 256, 2), (1, 16, 16, 1), (3, 32, 16, 4), (2, 64, 64, 32)]
+            (1, 48, 48, 8), (2, 192, 48, 8), (1, 256, 256, 2), (1, 16, 16, 1), (3, 32, 16, 4), (2, 64, 64, 32),
+            # bf16 with 16 l per tile: passes of 16 k (double-buffered), d = 64, one chunk of j
+            (1, 48, 48, 16), (2, 96, 64, 64), (1, 32, 16, 64)]
 
 
 @pytest.mark.parametrize("p", TC_CASES)
