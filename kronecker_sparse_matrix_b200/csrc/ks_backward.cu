@@ -29,6 +29,19 @@ namespace {
 __device__ __forceinline__ float ld_f(const float *p) { return __ldg(p); }
 __device__ __forceinline__ float ld_f(const __nv_bfloat16 *p) { return __bfloat162float(p[0]); }
 __device__ __forceinline__ void st_f(float *p, float v) { *p = v; }
+// the VEC = 16 / sizeof(T) elements of one 16-byte unit, as floats
+__device__ __forceinline__ void unpack16(const uint4 &w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y); f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 &w, float (&f)[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[h]));
+        f[2 * h] = t.x;
+        f[2 * h + 1] = t.y;
+    }
+}
 __device__ __forceinline__ void st_f(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
 
 // vt[i][l][j][k] = v[i][l][k][j]: 32 x 32 tiles of each b x c block through
@@ -66,7 +79,10 @@ __global__ void __launch_bounds__(256) transpose_blocks_kernel(const T *__restri
 // thread 8 k x 16 j fp32 sums, updated per row n with fma.rn.f32x2 on pairs of
 // j.  Stages of kNR rows of dY and X (the needed (k, l) and (j, l) runs) are
 // staged through registers into shared memory as [n][l][k] and [n][l][j],
-// the next stage's loads in flight while the current one computes.
+// the next stage's loads in flight while the current one computes.  With VEC
+// (the DL values of l of one k or j are whole 16-byte units: bf16 with DL = 8,
+// fp32 with DL = 4, 8, and 16-byte-aligned buffers) a thread loads 16-byte
+// units; otherwise one element at a time.
 constexpr int kDvThreads = 256;
 constexpr int kNR = 8;  // rows per stage
 
@@ -96,10 +112,15 @@ struct DvParams {
     long long vsize;      // a*b*c*d
 };
 
-template <typename T, int DL>
+template <typename T, int DL, bool VEC>
 __global__ void __launch_bounds__(kDvThreads, 1) dv_kernel(const DvParams p) {
     using TL = DvTile<DL>;
     constexpr int BK = TL::BK, BJ = TL::BJ;
+    constexpr int EV = 16 / (int)sizeof(T);  // elements per 16-byte unit
+    constexpr int UPR = VEC ? DL / EV : 1;   // units per (row, k) or (row, j)
+    // 16-byte units per thread and stage: e = (row, k, unit of l), unit fastest
+    constexpr int NAV = VEC ? (kNR * BK * UPR + kDvThreads - 1) / kDvThreads : 1;
+    constexpr int NBV = VEC ? (kNR * BJ * UPR + kDvThreads - 1) / kDvThreads : 1;
     extern __shared__ __align__(16) float dsm[];
     const T *dY = static_cast<const T *>(p.dY);
     const T *X = static_cast<const T *>(p.X);
@@ -122,9 +143,32 @@ __global__ void __launch_bounds__(kDvThreads, 1) dv_kernel(const DvParams p) {
     const int n_stages = (int)((n_end - n_begin + kNR - 1) / kNR);
 
     // staging roles: element e of a stage = (row, k or j, l), l fastest
-    float ra[TL::NA], rb[TL::NB];
+    float ra[VEC ? 1 : TL::NA], rb[VEC ? 1 : TL::NB];
+    uint4 va[NAV], vb[NBV];
     auto load_stage = [&](int s) {
         const long long nb = n_begin + (long long)s * kNR;
+        if constexpr (VEC) {
+#pragma unroll
+            for (int u = 0; u < NAV; ++u) {
+                const int e = tid + u * kDvThreads;
+                const int lu = e % UPR, k = (e / UPR) % BK, r = e / (UPR * BK);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (r < kNR && nb + r < n_end && k0 + k < p.b)
+                    v = __ldg(reinterpret_cast<const uint4 *>(dY + (nb + r) * p.out_f + (long long)i * p.b * p.d +
+                                                              (long long)(k0 + k) * p.d + l0 + lu * EV));
+                va[u] = v;
+            }
+#pragma unroll
+            for (int u = 0; u < NBV; ++u) {
+                const int e = tid + u * kDvThreads;
+                const int lu = e % UPR, j = (e / UPR) % BJ, r = e / (UPR * BJ);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (r < kNR && nb + r < n_end && j0 + j < p.c)
+                    v = __ldg(reinterpret_cast<const uint4 *>(X + (nb + r) * p.in_f + (long long)i * p.c * p.d +
+                                                              (long long)(j0 + j) * p.d + l0 + lu * EV));
+                vb[u] = v;
+            }
+        } else {
 #pragma unroll
         for (int u = 0; u < TL::NA; ++u) {
             const int e = tid + u * kDvThreads;
@@ -143,10 +187,35 @@ __global__ void __launch_bounds__(kDvThreads, 1) dv_kernel(const DvParams p) {
                 v = ld_f(X + (nb + r) * p.in_f + (long long)i * p.c * p.d + (long long)(j0 + j) * p.d + l0 + l);
             rb[u] = v;
         }
+        }
     };
     auto store_stage = [&](int buf) {
         float *sa = dsm + buf * (TL::SA + TL::SB);
         float *sb = sa + TL::SA;
+        if constexpr (VEC) {
+#pragma unroll
+            for (int u = 0; u < NAV; ++u) {
+                const int e = tid + u * kDvThreads;
+                const int lu = e % UPR, k = (e / UPR) % BK, r = e / (UPR * BK);
+                if (r < kNR) {
+                    float f[EV];
+                    unpack16(va[u], f);
+#pragma unroll
+                    for (int h = 0; h < EV; ++h) sa[(r * DL + lu * EV + h) * TL::KP + k] = f[h];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < NBV; ++u) {
+                const int e = tid + u * kDvThreads;
+                const int lu = e % UPR, j = (e / UPR) % BJ, r = e / (UPR * BJ);
+                if (r < kNR) {
+                    float f[EV];
+                    unpack16(vb[u], f);
+#pragma unroll
+                    for (int h = 0; h < EV; ++h) sb[(r * DL + lu * EV + h) * TL::JP + j] = f[h];
+                }
+            }
+        } else {
 #pragma unroll
         for (int u = 0; u < TL::NA; ++u) {
             const int e = tid + u * kDvThreads;
@@ -158,6 +227,7 @@ __global__ void __launch_bounds__(kDvThreads, 1) dv_kernel(const DvParams p) {
             const int e = tid + u * kDvThreads;
             const int l = e % DL, j = (e / DL) % BJ, r = e / (DL * BJ);
             if (r < kNR) sb[(r * DL + l) * TL::JP + j] = rb[u];
+        }
         }
     };
 
@@ -231,8 +301,18 @@ __global__ void __launch_bounds__(256) dv_reduce_kernel(const float *__restrict_
     }
 }
 
+template <typename T>
+cudaError_t launch_dv_reduce(const DvProblem &q, float *W, int splits) {
+    const long long vsize = q.a * q.b * q.c * q.d;
+    const long long rb = std::min<long long>((vsize + 255) / 256, (long long)sm_count() * 8);
+    dv_reduce_kernel<T><<<(int)std::max<long long>(rb, 1), 256, 0, q.stream>>>(W, static_cast<T *>(q.dV), vsize,
+                                                                               splits);
+    return cudaGetLastError();
+}
+
 template <typename T, int DL>
 cudaError_t launch_dv_typed(const DvProblem &q, float *W, int splits, long long rows_per_split) {
+    constexpr int EV = 16 / (int)sizeof(T);
     using TL = DvTile<DL>;
     DvParams p;
     p.dY = q.dY;
@@ -249,15 +329,15 @@ cudaError_t launch_dv_typed(const DvProblem &q, float *W, int splits, long long 
     p.vsize = q.a * q.b * q.c * q.d;
     const long long grid = (long long)p.n_g * p.n_kb * p.n_jb * splits;
     if (grid > INT32_MAX) return cudaErrorInvalidConfiguration;
-    auto kern = dv_kernel<T, DL>;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(q.dY) | reinterpret_cast<uintptr_t>(q.X)) % 16) == 0;
+    auto kern = dv_kernel<T, DL, false>;
+    if constexpr (DL % EV == 0)
+        if (aligned) kern = dv_kernel<T, DL, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<(int)grid, kDvThreads, TL::SMEM, q.stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const long long rb = std::min<long long>((p.vsize + 255) / 256, (long long)sm_count() * 8);
-    dv_reduce_kernel<T><<<(int)std::max<long long>(rb, 1), 256, 0, q.stream>>>(W, static_cast<T *>(q.dV), p.vsize,
-                                                                               splits);
-    return cudaGetLastError();
+    return launch_dv_reduce<T>(q, W, splits);
 }
 
 template <typename T>
@@ -335,6 +415,10 @@ cudaError_t launch_colsum(const void *dY, void *db, long long batch, long long w
 int dv_dl(int64_t d) { return d % 8 == 0 ? 8 : d % 4 == 0 ? 4 : d % 2 == 0 ? 2 : 1; }
 
 void dv_split(const DvProblem &q, int *splits, long long *rows_per_split) {
+    if (dv_tc_supported(q)) {
+        dv_tc_split(q, splits, rows_per_split);
+        return;
+    }
     const int dl = dv_dl(q.d);
     const int bk = 64 * (dl == 8 ? 1 : dl == 1 ? 4 : 2), bj = 64 * ((dl == 2 || dl == 1) ? 2 : 1);
     const long long tiles = q.a * (q.d / dl) * ((q.b + bk - 1) / bk) * ((q.c + bj - 1) / bj);
@@ -349,6 +433,10 @@ void dv_split(const DvProblem &q, int *splits, long long *rows_per_split) {
 }
 
 cudaError_t launch_dv(const DvProblem &q, float *W, int splits, long long rows_per_split) {
+    if (dv_tc_supported(q)) {  // tensor cores for the partial sums, then the same ordered reduction
+        cudaError_t e = launch_dv_tc(q, W, splits, rows_per_split);
+        return e != cudaSuccess ? e : launch_dv_reduce<__nv_bfloat16>(q, W, splits);
+    }
     if (q.dtype == KS_BF16) return launch_dv_dl<__nv_bfloat16>(q, W, splits, rows_per_split);
     return launch_dv_dl<float>(q, W, splits, rows_per_split);
 }

@@ -83,6 +83,13 @@ struct DvProblem {
 int dv_dl(int64_t d);
 void dv_split(const DvProblem &q, int *splits, long long *rows_per_split);
 cudaError_t launch_dv(const DvProblem &q, float *W, int splits, long long rows_per_split);
+// dV on the tensor cores (ks_dv_tc.cu): bf16, d % 8 == 0, c % 16 == 0, c <= 64,
+// b >= 128, 16-byte-aligned buffers; row ranges are multiples of 16.
+bool dv_tc_supported(const DvProblem &q);
+void dv_tc_split(const DvProblem &q, int *splits, long long *rows_per_split);
+cudaError_t launch_dv_tc(const DvProblem &q, float *W, int splits, long long rows_per_split);
+// The driver's cuTensorMapEncodeTiled (ks_tc.cu), or null when unavailable.
+void *tensor_map_encoder();
 // Column sums db[col] = sum_n dY[n][col] (ks_backward.cu): fp32 partial sums
 // over `splits` row ranges into W[split][width], then added in range order.
 void colsum_split(long long batch, long long width, int *splits, long long *rows_per_split);

@@ -1004,6 +1004,8 @@ static cudaError_t launch_typed(const Problem &p, const TcConfig &cfg) {
     }
 }
 
+void *tensor_map_encoder() { return reinterpret_cast<void *>(encode_fn()); }
+
 cudaError_t launch_tc(const Problem &p, const TcConfig &cfg) {
     if (p.dtype == KS_BF16) return launch_typed<__nv_bfloat16>(p, cfg);
     if (p.dtype == KS_TF32) return launch_typed<float>(p, cfg);

@@ -54,6 +54,40 @@ def test_dv_matches_oracle(p, dtype):
         assert oracle.max_rel_err(dv.cpu().reshape(-1), oracle.dv(dy, X, p)) <= TOL[dtype], (p, batch)
 
 
+# bf16 patterns that take the tensor-core dV kernel (d % 8 == 0, c % 16 == 0 up to
+# 64, b >= 128): one and several 128-k tiles (b = 160: a tail of 32 k), one and
+# three groups of 8 l, several blocks, c = 16 .. 64.
+DV_TC_PATTERNS = [(1, 256, 64, 16), (2, 128, 32, 8), (1, 160, 16, 24), (3, 128, 64, 8), (1, 192, 48, 8)]
+
+
+def cuda_kernel_names(fn):
+    with torch.profiler.profile(activities=[torch.profiler.ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return {e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA}
+
+
+@pytest.mark.parametrize("p", DV_TC_PATTERNS)
+def test_dv_tensor_core_path_matches_oracle(p):
+    for batch in (1, 9, 300, 1111):
+        X, V, dy = grad_inputs(p, batch, torch.bfloat16, seed=sum(p) + 5 * batch)
+        dv = ks.matmul_dv(dy.to(DEV), X.to(DEV), p)
+        ks.sync_status()
+        assert oracle.max_rel_err(dv.cpu().reshape(-1), oracle.dv(dy, X, p)) <= TOL[torch.bfloat16], (p, batch)
+
+
+def test_dv_tensor_core_path_full_gpt2_batch():
+    f = inputs.gpt2(dtype=torch.bfloat16, device=DEV)
+    p = f.pattern
+    g = torch.Generator(device=DEV).manual_seed(6)
+    dy = torch.randn(f.batch, inputs.out_features(p), generator=g, device=DEV).to(torch.bfloat16)
+    names = cuda_kernel_names(lambda: ks.matmul_dv(dy, f.X, p))
+    assert any("dv_tc_kernel" in n for n in names), names
+    dv = ks.matmul_dv(dy, f.X, p)
+    ks.sync_status()
+    assert oracle.max_rel_err(dv.cpu().reshape(-1), oracle.dv(dy.cpu(), f.X.cpu(), p)) <= TOL[torch.bfloat16]
+
+
 def test_dv_full_vit_batch():
     f = inputs.vit(device=DEV)
     p = f.pattern

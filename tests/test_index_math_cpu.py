@@ -316,6 +316,56 @@ def test_tc_bf16_dls16_mma_descriptor_reads_what_the_transposer_wrote():
             assert q * 16 == (j * 16 + 8 * h) * 2
 
 
+# ------------------------------------------------------------- ks_dv_tc.cu
+def dv_tc_transposer(mn_rows):
+    """The bf16 dV kernel's transposer for one operand of a stage (16 rows n):
+    raw [n][mn][8 l] (16-byte unit = 8 l) -> per-l K-major planes with the
+    32-byte swizzle, row mn = 32 bytes (16 n), half h of row mn at
+    h ^ bit 2 of mn.  Task = (mn, row half nh) for tasks t < 2 * mn_rows
+    (A: t = thread + 128 nh, mn = thread; B: mn = t % c, nh = t // c).
+    Returns per task its raw read addresses (8 units) and its 8 writes (l)."""
+    plane = mn_rows * 32
+    out = {}
+    for t in range(2 * mn_rows):
+        mn, nh = (t % 128, t // 128) if mn_rows == 128 else (t % mn_rows, t // mn_rows)
+        reads = [((8 * nh + r) * mn_rows + mn) * 16 for r in range(8)]
+        writes = [e * plane + mn * 32 + ((nh ^ ((mn >> 2) & 1)) << 4) for e in range(8)]
+        out[t] = (mn, nh, reads, writes)
+    return out
+
+
+@pytest.mark.parametrize("mn_rows", [128, 64, 48, 32, 16])
+def test_dv_tc_transposer_is_in_place_and_matches_the_k_major_descriptor(mn_rows):
+    """Both operands of the dV kernel: every raw unit read once, every plane
+    unit written once inside the raw stage, quarter-warps reach eight bank
+    groups on reads (and on writes except where a quarter-warp straddles the
+    row halves of a narrow operand), and the K-major 32-byte-swizzle
+    descriptor (SBO = 256 bytes) reads X[n][mn][l] at element (mn, n)."""
+    tr = dv_tc_transposer(mn_rows)
+    raw = 16 * mn_rows * 16
+    reads = sorted(a for v in tr.values() for a in v[2])
+    writes = sorted(a for v in tr.values() for a in v[3])
+    assert reads == list(range(0, raw, 16)) and writes == list(range(0, raw, 16))
+    for t0 in range(0, len(tr), 8):
+        q = [tr[t] for t in range(t0, min(t0 + 8, len(tr)))]
+        for r in range(8):
+            assert len({(v[2][r] // 16) % 8 for v in q}) == len(q)
+        if all(v[1] == q[0][1] for v in q):
+            for e in range(8):
+                assert len({(v[3][e] // 16) % 8 for v in q}) == len(q)
+    where = {}
+    for mn, nh, rd, wr in tr.values():
+        for e in range(8):
+            for h in range(8):
+                where[(mn, 8 * nh + h, e)] = wr[e] + 2 * h
+    for l in range(8):
+        for mn in range(mn_rows):
+            for k in range(16):
+                a = mn * 32 + (k // 8) * 16 + (k % 8) * 2
+                a ^= ((a >> 7) & 1) << 4  # the 32-byte swizzle: bit 4 ^= bit 7
+                assert l * mn_rows * 32 + a == where[(mn, k, l)]
+
+
 def tf32_tasks(dls):
     """The fp32 transposer of ks_tc.cu, modelled per thread t (0..127) and task
     k: the raw addresses it reads (one list per load instruction) and, per
