@@ -27,8 +27,9 @@
 //   warp 1      one thread issues per l one MMA (M = 128, N = c, K = 16) into
 //               TMEM columns l*c .. l*c + c - 1.
 // After the last stage warps 2..5 read the accumulators (warp w: TMEM lanes
-// 32 (w % 4) ..) and store the partial sums.  Every mbarrier wait is bounded;
-// a wait that runs out sets the device status word and ends every role.
+// 32 (w % 4) ..) and store the partial sums.  Every mbarrier wait is bounded
+// (about one second, or at once under KS_FAULT_INJECT=timeout); a wait that
+// runs out sets the device status word and ends every role.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -57,6 +58,7 @@ struct DvTcParams {
     int b, c, d;
     int n_g, n_kt;
     unsigned *status;
+    unsigned long long wait_ns;  // bound of the pipeline's waits
 };
 
 __global__ void __launch_bounds__(kDvThreads, 1)
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kDvThreads, 1)
             int s = 0;
             for (; s < n_stages && ok; ++s) {
                 const int slot = s % kDvStages;
-                ok = mbar_wait(&x_empty[slot], ((s / kDvStages) & 1) ^ 1, abort_flag, p.status);
+                ok = mbar_wait(&x_empty[slot], ((s / kDvStages) & 1) ^ 1, abort_flag, p.status, p.wait_ns);
                 if (!ok) break;
                 uint8_t *st = smem + slot * stage_bytes;
                 const int n0 = (int)(n_begin + (long long)s * kDvRows);
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(kDvThreads, 1)
             bool ok = true;
             for (int s = 0; s < n_stages && ok; ++s) {
                 const int slot = s % kDvStages;
-                ok = mbar_wait(&a_ready[slot], (s / kDvStages) & 1, abort_flag, p.status);
+                ok = mbar_wait(&a_ready[slot], (s / kDvStages) & 1, abort_flag, p.status, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sa = su32(smem + slot * stage_bytes), sb = sa + (uint32_t)a_bytes;
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kDvThreads, 1)
         bool ok = true;
         for (int s = 0; s < n_stages && ok; ++s) {
             const int slot = s % kDvStages;
-            const bool w = mbar_wait(&x_full[slot], (s / kDvStages) & 1, abort_flag, p.status);
+            const bool w = mbar_wait(&x_full[slot], (s / kDvStages) & 1, abort_flag, p.status, p.wait_ns);
             ok = bar_and(1, 128, w);  // uniform over the four warps
             if (!ok) break;
             uint8_t *st = smem + slot * stage_bytes;
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kDvThreads, 1)
             mbar_arrive(&a_ready[slot]);
         }
         // epilogue: this warp's 32 TMEM lanes are k = k0 + 32 (warp % 4) + lane
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status, p.wait_ns));
         if (ok && n_stages > 0) {
             tc_fence_after();
             const int quad = warp & 3;
@@ -285,6 +287,7 @@ cudaError_t launch_dv_tc(const DvProblem &q, float *W, int splits, long long row
     p.n_kt = (int)((q.b + kDvM - 1) / kDvM);
     p.status = device_status_ptr();
     if (!p.status) return cudaErrorUnknown;
+    p.wait_ns = pipeline_wait_bound_ns();
     const int stage_bytes = kDvRows * (kDvM + (int)q.c) * 16;
     const int smem = kDvStages * stage_bytes + 3 * kDvStages * 8 + 8 + 16 + 1024;
     const long long grid = (long long)p.n_g * p.n_kt * splits;

@@ -90,6 +90,9 @@ void dv_tc_split(const DvProblem &q, int *splits, long long *rows_per_split);
 cudaError_t launch_dv_tc(const DvProblem &q, float *W, int splits, long long rows_per_split);
 // The driver's cuTensorMapEncodeTiled (ks_tc.cu), or null when unavailable.
 void *tensor_map_encoder();
+// Bound of the tensor-core pipelines' mbarrier waits in ns (ks_tc.cu): about
+// one second, or 0 under KS_FAULT_INJECT=timeout.
+unsigned long long pipeline_wait_bound_ns();
 // Column sums db[col] = sum_n dY[n][col] (ks_backward.cu): fp32 partial sums
 // over `splits` row ranges into W[split][width], then added in range order.
 void colsum_split(long long batch, long long width, int *splits, long long *rows_per_split);

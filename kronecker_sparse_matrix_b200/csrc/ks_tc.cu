@@ -822,14 +822,14 @@ bool tc_layout(int dls, int bp, int es, bool bias, TcLayout *out) {
     return true;
 }
 
-// KS_FAULT_INJECT=timeout: the pipeline's waits give up at once (tests of the
-// device status word); otherwise about one second.
-unsigned long long tc_wait_bound_ns() {
-    const char *f = getenv("KS_FAULT_INJECT");
-    return (f && strcmp(f, "timeout") == 0) ? 0ull : (unsigned long long)kTimeoutNs;
-}
-
 }  // namespace
+
+// KS_FAULT_INJECT=timeout: the tensor-core pipelines' waits give up at once
+// (tests of the device status word); otherwise about one second.
+unsigned long long pipeline_wait_bound_ns() {
+    const char *f = getenv("KS_FAULT_INJECT");
+    return (f && strcmp(f, "timeout") == 0) ? 0ull : (unsigned long long)sm100::kTimeoutNs;
+}
 
 TcConfig tc_choose(const Problem &p) {
     const int dls = tc_dls(p);
@@ -972,7 +972,7 @@ static cudaError_t launch_dls(const Problem &pr, const TcConfig &cfg) {
     p.Y = pr.Y;
     p.status = device_status_ptr();
     if (!p.status) return cudaErrorUnknown;
-    p.wait_ns = tc_wait_bound_ns();
+    p.wait_ns = pipeline_wait_bound_ns();
     p.stages = L.stages;
     p.vstages = L.vstages;
     p.off_v = L.off_v;

@@ -5,11 +5,12 @@ entry point that needs a workspace returns KS_ERR_ALLOC before it launches
 anything, so its output is left as it was; ks_matmul, whose fp32 workspace is
 optional, reads the values in place and is still correct.
 
-KS_FAULT_INJECT=timeout makes the tensor-core kernel's pipeline waits give up
-at once: the kernel abandons its tile loop, drains its in-flight copies and
-MMAs (bounded), frees its tensor memory and returns, and ks_sync_status
-reports KS_ERR_TIMEOUT.  The context stays usable: the next call on the same
-stream is checked against the oracle.
+KS_FAULT_INJECT=timeout makes the tensor-core kernels' pipeline waits give up
+at once (the forward product and the bf16 values gradient): the kernel
+abandons its loop, drains its in-flight copies and MMAs (bounded), frees its
+tensor memory and returns, and ks_sync_status reports KS_ERR_TIMEOUT.  The
+context stays usable: the next call on the same stream is checked against the
+oracle.
 """
 import numpy as np
 import pytest
@@ -111,3 +112,21 @@ def test_tc_wait_timeout_is_reported_and_the_next_call_is_correct(monkeypatch, p
     ks.sync_status()
     tol = 5e-3 if tf32 else 1e-2
     assert oracle.max_rel_err(Y.cpu(), oracle.matmul(f.X.cpu(), f.values.cpu(), p)) <= tol
+
+
+def test_dv_tensor_core_wait_timeout_is_reported_and_the_next_call_is_correct(monkeypatch):
+    p = (1, 256, 64, 16)  # bf16 dV on the tensor cores
+    f = inputs.factor_inputs(p, 300, seed=17, dtype=torch.bfloat16, device=DEV)
+    dy = torch.randn(300, inputs.out_features(p), generator=torch.Generator(device=DEV).manual_seed(18),
+                     device=DEV).to(torch.bfloat16)
+    ks.sync_status()
+    monkeypatch.setenv("KS_FAULT_INJECT", "timeout")
+    ks.matmul_dv(dy, f.X, p)  # the launches themselves succeed
+    with pytest.raises(ks.KsError) as err:
+        ks.sync_status()
+    assert err.value.status == 6
+    ks.sync_status()
+    monkeypatch.delenv("KS_FAULT_INJECT")
+    dv = ks.matmul_dv(dy, f.X, p)
+    ks.sync_status()
+    assert oracle.max_rel_err(dv.cpu().reshape(-1), oracle.dv(dy.cpu(), f.X.cpu(), p)) <= 1e-2
