@@ -175,11 +175,13 @@ ks_status ks_matmul_dx(const void *dY, const void *values, int64_t a, int64_t b,
  *     dV[i][l][k][j] = sum_{n<batch} dY[n][i*b*d + k*d + l] * X[n][i*c*d + j*d + l],
  * written (not accumulated) in the values layout [a][d][b][c].  dY is
  * batch x (a*b*d), X batch x (a*c*d); DEVICE pointers of one dtype, dV must
- * not overlap dY or X.  Sums are fp32: each CTA sums a range of rows in row
- * order, and the partial sums of the ranges (a stream-ordered fp32 workspace
- * from the library's pool, at most 256 MiB) are added in range order, so the
- * result is deterministic; bf16 dV is rounded once at the end.  batch == 0
- * writes zeros. */
+ * not overlap dY or X.  Sums are fp32 over ranges of rows: on CUDA cores in
+ * row order, or, for bf16 with d % 8 == 0, c % 16 == 0 up to 64, b >= 128 and
+ * 16-byte-aligned dY and X, on the tensor cores in steps of 16 rows.  The
+ * partial sums of the ranges (a stream-ordered fp32 workspace from the
+ * library's pool, at most 256 MiB; KS_ERR_ALLOC if it cannot be had) are added
+ * in range order, so the result is deterministic; bf16 dV is rounded once at
+ * the end.  batch == 0 writes zeros. */
 ks_status ks_matmul_dv(const void *dY, const void *X, int64_t a, int64_t b,
                        int64_t c, int64_t d, int64_t batch, void *dV, int dtype,
                        void *stream);
@@ -310,11 +312,13 @@ ks_status ks_fma_rate_probe(float *out, int blocks, int64_t iters, void *stream)
  *                            points that need one return KS_ERR_ALLOC before
  *                            launching anything (ks_matmul reads the values in
  *                            place instead);
- *   KS_FAULT_INJECT=timeout  the tensor-core kernel's pipeline waits give up at
- *                            once instead of after about one second: the kernel
- *                            abandons its work (Y is unspecified), drains its
- *                            copies, frees its tensor memory and returns, and
- *                            the next ks_sync_status reports KS_ERR_TIMEOUT.
+ *   KS_FAULT_INJECT=timeout  the tensor-core kernels' pipeline waits (the
+ *                            product's and the bf16 dV's) give up at once
+ *                            instead of after about one second: the kernel
+ *                            abandons its work (its output is unspecified),
+ *                            drains its copies, frees its tensor memory and
+ *                            returns, and the next ks_sync_status reports
+ *                            KS_ERR_TIMEOUT.
  * Unset (or any other value), nothing is injected. */
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
