@@ -42,6 +42,24 @@ def test_fused_epilogue(case, act):
     assert oracle.max_rel_err(Y.cpu(), ref) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("p,dtype,variant", [((1, 48, 48, 8), torch.float32, "fma"),
+                                               ((2, 64, 32, 4), torch.float32, "fma"),
+                                               ((1, 192, 48, 8), torch.bfloat16, "auto")])
+def test_bias_not_16_byte_aligned(p, dtype, variant):
+    # a bias view one element into its buffer: the fp32 kernel reads it one
+    # element at a time, and the tensor-core kernel (which needs a 16-byte
+    # aligned bias) is not chosen, so the CUDA-core kernel runs the product
+    f = inputs.factor_inputs(p, 131, seed=9, dtype=dtype)
+    g = torch.Generator().manual_seed(4)
+    buf = torch.randn(inputs.out_features(p) + 1, generator=g).to(dtype).to(DEV)
+    bias = buf[1:]
+    assert bias.data_ptr() % 16 != 0
+    Y = ks.matmul(f.X.to(DEV), f.values.to(DEV), p, variant=variant, bias=bias, act="gelu_tanh")
+    ks.sync_status()
+    ref = oracle.matmul_epilogue(f.X, f.values, p, bias.cpu(), "gelu_tanh")
+    assert oracle.max_rel_err(Y.cpu(), ref) <= TOL[dtype]
+
+
 @pytest.mark.parametrize("act", ["relu", "gelu_erf"])
 def test_activation_without_bias(act):
     p = (1, 48, 48, 8)
