@@ -119,7 +119,8 @@ ks_status ks_matmul(const void *X, const void *values, int64_t a, int64_t b,
 /* ks_matmul for a batch that lives in HOST memory: X (batch x a*c*d),
  * values and Y (batch x a*b*d) are HOST pointers, laid out as for ks_matmul.
  * The library copies the values to the device once and streams the rows
- * through in chunks (about six, each a multiple of 128 rows, at least 1024):
+ * through in chunks (1 to 32, more for larger batches, each a multiple of
+ * 128 rows):
  * the copy of chunk k+1 to the device, the product of chunk k and the copy of
  * chunk k-1 back to the host run at the same time, on three streams the
  * library keeps per device, ordered after earlier work on `stream`; `stream`
