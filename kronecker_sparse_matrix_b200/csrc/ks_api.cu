@@ -343,7 +343,7 @@ ks_status ks_chain_ep(const void *X, const void *const *factors, const ks_patter
             if (ranges_overlap(Y, width, factors[t], 4096 * 2 * (int64_t)elem))
                 return fail(KS_ERR_INVALID_ARG, "Y overlaps factor %d", t);
         if (butterfly12_supported(X, factors, Y, dtype)) {
-            const cudaError_t e = launch_butterfly12(X, factors, batch, Y, dtype, 8, st);
+            const cudaError_t e = launch_butterfly12(X, factors, batch, Y, dtype, st);
             if (e != cudaSuccess) return cuda_fail(e, "fused butterfly chain launch");
             return ok();
         }

@@ -16,9 +16,16 @@
 // pass a thread owns the 16 entries that differ in that digit, for R rows, in
 // registers, and applies four factors there.  Between passes the rows go
 // through shared memory in an XOR-swizzled order in which all three thread
-// mappings are free of bank conflicts.  X is read once and Y written once;
-// each pair's 2 x 2 weights are loaded once per R rows (from L2, where the
-// 12 x 2048 pairs stay resident).
+// mappings are free of bank conflicts.  X is read once and Y written once.
+//
+// Weights.  In passes 1 and 2 a warp's lanes take consecutive pairs, so each
+// weight load is coalesced; they come from L2 (where the 12 x 2048 pairs stay)
+// once per R rows.  In pass 3 the eight pairs of a thread are one contiguous
+// line and a warp's load would touch 32 lines, so factors 9-12 are copied once
+// per CTA into shared memory as fp32, line t (the thread's) with its eight
+// 16-byte slots rotated by t & 7: both the coalesced copy and the per-thread
+// reads are then free of bank conflicts.  (Keeping bf16 weights as bf16 there,
+// with 8 rows per block, measured slower.)
 //
 // Rounding: fp32 FMAs, y = fma(V[k][1], x1, V[k][0] * x0), intermediates kept
 // in fp32 (bf16 chains round only the final output).
@@ -97,6 +104,25 @@ __device__ __forceinline__ void apply_factor(float (&v)[R][16], const T *V, int 
     }
 }
 
+// Pass-3 factor from the resident copy: the k-th pair of thread t at slot
+// k ^ tx of line t (tx = t & 7).
+template <int R, int S>
+__device__ __forceinline__ void apply_factor_res(float (&v)[R][16], const float4 *line, int tx) {
+    int k = 0;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        if (m & (1 << S)) continue;
+        const float4 w = line[k ^ tx];
+        ++k;
+        const int m1 = m | (1 << S);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float x0 = v[r][m], x1 = v[r][m1];
+            v[r][m] = fmaf(w.y, x1, w.x * x0);
+            v[r][m1] = fmaf(w.w, x1, w.z * x0);
+        }
+    }
+}
 // Shared-memory position of entry e = (A, B, C) digits (bits 11-8, 7-4, 3-0):
 //   A*256 + ((B ^ A) & 15) * 16 + (C ^ ((B >> 1) | (A & 1) << 3)),
 // a bijection on 0..4095 under which, for every pass's thread mapping, the 32
@@ -107,8 +133,9 @@ __device__ __forceinline__ int swz(int e) {
 }
 
 template <typename T, int R>
-__global__ void __launch_bounds__(kThreads, R <= 4 ? 2 : 1) butterfly12_kernel(const BflyParams p) {
-    extern __shared__ float sm[];  // R rows of 4096 fp32 in swizzled order
+__global__ void __launch_bounds__(kThreads, 1) butterfly12_kernel(const BflyParams p) {
+    // R rows of 4096 fp32 in swizzled order, then factors 9-12's weights
+    extern __shared__ float sm[];
     const T *X = static_cast<const T *>(p.X);
     T *Y = static_cast<T *>(p.Y);
     const int t = threadIdx.x;
@@ -125,11 +152,24 @@ __global__ void __launch_bounds__(kThreads, R <= 4 ? 2 : 1) butterfly12_kernel(c
     // Weight index bases (q without the digit's contribution).
     const int q1 = t;                                 // pass 1: bits 7-0 stay below p
     const int q2 = ((t >> 4) << 7) | (t & 15);        // pass 2: A moves down one bit
-    const int q3 = t << 3;                            // pass 3: A, B move down one bit
     const T *V[12];
 #pragma unroll
     for (int k = 0; k < 12; ++k) V[k] = static_cast<const T *>(p.V[k]);
 
+    // factors 9-12 into shared memory: pair g of factor f (g = t + 256 i, read
+    // coalesced) goes to line g >> 3, slot (g & 7) ^ (line & 7); a thread's
+    // reads in pass 3 are then conflict-free (lines are its own, slots rotate)
+    float4 *res = reinterpret_cast<float4 *>(sm + R * kWidth);
+#pragma unroll
+    for (int f = 0; f < 4; ++f)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int g = t + 256 * i, line = g >> 3;
+            res[f * 2048 + line * 8 + ((g & 7) ^ (line & 7))] = BflyIO<T>::weights(V[8 + f], g);
+        }
+    // (the first pass-1 -> pass-2 barrier orders these stores before any read)
+    const float4 *res_t = res + t * 8;
+    const int tx = t & 7;
     const long long n_blocks = (p.N + R - 1) / R;
     for (long long blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
         const long long n0 = blk * R;
@@ -171,10 +211,10 @@ __global__ void __launch_bounds__(kThreads, R <= 4 ? 2 : 1) butterfly12_kernel(c
         for (int r = 0; r < R; ++r)
 #pragma unroll
             for (int C = 0; C < 16; ++C) v[r][C] = sm[r * kWidth + (u3 ^ C)];
-        apply_factor<T, R, 0, 3>(v, V[8], q3);
-        apply_factor<T, R, 0, 2>(v, V[9], q3);
-        apply_factor<T, R, 0, 1>(v, V[10], q3);
-        apply_factor<T, R, 0, 0>(v, V[11], q3);
+        apply_factor_res<R, 3>(v, res_t, tx);
+        apply_factor_res<R, 2>(v, res_t + 2048, tx);
+        apply_factor_res<R, 1>(v, res_t + 4096, tx);
+        apply_factor_res<R, 0>(v, res_t + 6144, tx);
 #pragma unroll
         for (int r = 0; r < R; ++r)
             if (n0 + r < p.N) BflyIO<T>::store16(Y + (n0 + r) * kWidth + (t << 4), v[r]);
@@ -184,12 +224,12 @@ __global__ void __launch_bounds__(kThreads, R <= 4 ? 2 : 1) butterfly12_kernel(c
 
 template <typename T, int R>
 cudaError_t launch_bfly(const BflyParams &p, cudaStream_t stream) {
-    const size_t smem = (size_t)R * kWidth * sizeof(float);
+    const size_t smem = (size_t)R * kWidth * sizeof(float) + 4 * 2048 * sizeof(float4);
     auto kern = butterfly12_kernel<T, R>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long n_blocks = (p.N + R - 1) / R;
-    const long long grid = std::min<long long>(n_blocks, (long long)sm_count() * (R <= 4 ? 2 : 1));
+    const long long grid = std::min<long long>(n_blocks, (long long)sm_count());
     kern<<<(int)grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -215,15 +255,16 @@ bool butterfly12_supported(const void *X, const void *const *factors, void *Y, i
 }
 
 cudaError_t launch_butterfly12(const void *X, const void *const *factors, long long batch, void *Y, int dtype,
-                               int rows_per_block, cudaStream_t stream) {
+                               cudaStream_t stream) {
     BflyParams p;
     p.X = X;
     p.Y = Y;
     p.N = batch;
     for (int t = 0; t < 12; ++t) p.V[t] = factors[t];
-    if (dtype == KS_BF16)
-        return rows_per_block == 8 ? launch_bfly<__nv_bfloat16, 8>(p, stream) : launch_bfly<__nv_bfloat16, 4>(p, stream);
-    return rows_per_block == 8 ? launch_bfly<float, 8>(p, stream) : launch_bfly<float, 4>(p, stream);
+    // 6 rows per block: their 96 KB and the 128 KB of fp32 pass-3 weights fill
+    // the 227 KB of shared memory a CTA may take
+    if (dtype == KS_BF16) return launch_bfly<__nv_bfloat16, 6>(p, stream);
+    return launch_bfly<float, 6>(p, stream);
 }
 
 }  // namespace ks

@@ -125,7 +125,7 @@ ks_status matmul_no_workspace(const void *X, const void *V, int64_t a, int64_t b
 bool butterfly12_matches(const ks_pattern *patterns, int n);
 bool butterfly12_supported(const void *X, const void *const *factors, void *Y, int dtype);
 cudaError_t launch_butterfly12(const void *X, const void *const *factors, long long batch, void *Y, int dtype,
-                               int rows_per_block, cudaStream_t stream);
+                               cudaStream_t stream);
 
 // Device status word (ks_api.cu): kernels OR these bits in on failure.
 enum DeviceStatusBits : unsigned {

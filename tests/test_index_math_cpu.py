@@ -650,3 +650,55 @@ def test_tc_fused_bias_units_are_aligned_and_cover_the_chunk(es):
                         e0, lu = (rpu * u) // dls, (rpu * u) % dls
                         assert off == ybase + l0 + (ps * bp + oc * kc + e0) * d + lu
                         assert (off * es) % 16 == 0 and off + rpu <= a * b * d
+
+
+# ------------------------------------------------------------ ks_butterfly.cu
+def bfly_swz(e):
+    A, B, C = e >> 8, (e >> 4) & 15, e & 15
+    return (A << 8) | (((B ^ A) & 15) << 4) | (C ^ ((B >> 1) | ((A & 1) << 3)))
+
+
+def test_butterfly_row_order_is_a_bijection_and_every_pass_is_conflict_free():
+    assert sorted(bfly_swz(e) for e in range(4096)) == list(range(4096))
+    for t in range(256):
+        u1, u2, u3 = bfly_swz(t), bfly_swz(((t >> 4) << 8) | (t & 15)), bfly_swz(t << 4)
+        for D in range(16):
+            # the kernel's per-pass shortcuts equal the order of the entry each thread holds
+            assert (D << 8) | (u1 ^ ((D << 4) | ((D & 1) << 3))) == bfly_swz((D << 8) | t)
+            assert u2 ^ ((D << 4) | (D >> 1)) == bfly_swz(((t >> 4) << 8) | (D << 4) | (t & 15))
+            assert u3 ^ D == bfly_swz((t << 4) | D)
+    for w in range(8):
+        lanes = range(32 * w, 32 * w + 32)
+        for D in range(16):
+            for pas in ((lambda t: (D << 8) | t), (lambda t: ((t >> 4) << 8) | (D << 4) | (t & 15)),
+                        (lambda t: (t << 4) | D)):
+                assert wavefronts([bfly_swz(pas(t)) for t in lanes], 1) == 1
+
+
+def test_butterfly_resident_pass3_weights_cover_each_pair_and_are_conflict_free():
+    slot_words = 4                         # one float4 (a pair's 2 x 2 weights in fp32)
+    rot = lambda line: line & 7
+    rows = 6
+    assert rows * 4096 * 4 + 4 * 2048 * 4 * slot_words <= 232448
+    for f in range(4):
+        where = {}
+        for i in range(8):
+            for w in range(8):
+                addrs = []
+                for t in range(32 * w, 32 * w + 32):
+                    g = t + 256 * i
+                    idx = f * 2048 + (g >> 3) * 8 + ((g & 7) ^ rot(g >> 3))
+                    assert idx not in where.values()
+                    where[g] = idx
+                    addrs.append(idx * slot_words)
+                assert wavefronts(addrs, slot_words) == slot_words   # 512 or 256 bytes: optimal
+        assert sorted(where) == list(range(2048))
+        # pass 3: thread t's k-th pair (q = 8t + k) is read at slot k ^ rot(t) of line t
+        for k in range(8):
+            for w in range(8):
+                addrs = []
+                for t in range(32 * w, 32 * w + 32):
+                    idx = f * 2048 + t * 8 + (k ^ rot(t))
+                    assert where[8 * t + k] == idx
+                    addrs.append(idx * slot_words)
+                assert wavefronts(addrs, slot_words) == slot_words
