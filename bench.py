@@ -298,11 +298,11 @@ def rank_seed(seed, rank):
 # Source files of each kernel family: a recorded ncu traffic figure stays
 # valid only while these are unchanged.
 FAMILY_SOURCES = {
-    "fma-fp32": ["ks_fma32.cu", "ks_fma.cu", "ks_internal.h"],
-    "fma-bf16": ["ks_fma.cu", "ks_internal.h"],
-    "tc-bf16": ["ks_tc.cu", "ks_sm100.cuh", "ks_internal.h"],
-    "stream-fp32": ["ks_stream.cu", "ks_internal.h"],
-    "stream-bf16": ["ks_stream.cu", "ks_internal.h"],
+    "fma-fp32": ["ks_fma32.cu", "ks_fma.cu", "ks_internal.h", "ks_epilogue.cuh"],
+    "fma-bf16": ["ks_fma.cu", "ks_internal.h", "ks_epilogue.cuh"],
+    "tc-bf16": ["ks_tc.cu", "ks_sm100.cuh", "ks_internal.h", "ks_epilogue.cuh"],
+    "stream-fp32": ["ks_stream.cu", "ks_internal.h", "ks_epilogue.cuh"],
+    "stream-bf16": ["ks_stream.cu", "ks_internal.h", "ks_epilogue.cuh"],
 }
 
 

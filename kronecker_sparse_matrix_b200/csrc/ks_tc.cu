@@ -661,8 +661,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (EP && p.act) {
+                    if (p.act == 2) {
+                        static_assert(KCM % 2 == 0, "pairs of columns");
+                        // GELU, tanh form, two values per step in the packed fp32
+                        // instructions: u = z (c0 + c1 z^2) with c0 = sqrt(2/pi) and
+                        // c1 = 0.044715 c0, h = z / 2, h + h tanh(u) (the hardware
+                        // tanh).  The whole chunk in one block, so the scheduler can
+                        // interleave every element's chain: 1.23x on GPT-2 bf16 with
+                        // bias + GELU against one element at a time; the same
+                        // arithmetic split per l plane, or moved into a helper that
+                        // takes the tile, measured 1.0x and 1.06x.
 #pragma unroll
-                    for (int l = 0; l < DLS; ++l) ep_act_array_hw(acc[l], p.act);
+                        for (int l = 0; l < DLS; ++l) {
+#pragma unroll
+                            for (int e = 0; e + 1 < KCM; e += 2) {
+                                const float2 z = make_float2(acc[l][e], acc[l][e + 1]);
+                                const float2 z2 = __fmul2_rn(z, z);
+                                const float2 q = __ffma2_rn(z2, make_float2(0.0356774081f, 0.0356774081f),
+                                                            make_float2(0.7978845608f, 0.7978845608f));
+                                const float2 u = __fmul2_rn(z, q);
+                                const float2 h = __fmul2_rn(z, make_float2(0.5f, 0.5f));
+                                const float2 t = make_float2(tanh_hw(u.x), tanh_hw(u.y));
+                                const float2 y = __ffma2_rn(h, t, h);
+                                acc[l][e] = y.x;
+                                acc[l][e + 1] = y.y;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int l = 0; l < DLS; ++l) ep_act_array(acc[l], p.act);
+                    }
                 }
                 if (p.ytma) {  // the previous box store has finished reading the staging
                     if (lane == 0) bulk_wait_read_all();
