@@ -34,6 +34,10 @@
  *     call is asynchronous on that stream; the return value reports only
  *     errors found before or at launch.  Errors found on the device (a bounded
  *     wait that gave up) are reported by ks_sync_status().
+ *   - Calls run on the calling thread's current CUDA device; device buffers
+ *     and the stream must belong to it.  The library's per-device state
+ *     (workspace pool, status word, helper streams) is kept per device, so a
+ *     process may drive several GPUs by switching the current device.
  *   - Y must not overlap X or values (KS_ERR_INVALID_ARG).
  *   - batch == 0 is a no-op returning KS_OK.  Negative or zero pattern
  *     entries, negative batch, or sizes whose element counts overflow int64
