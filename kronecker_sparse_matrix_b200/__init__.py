@@ -21,7 +21,8 @@ from ._lib import (KS_BF16, KS_F32, KS_TF32, KS_VARIANT_AUTO, KS_VARIANT_FMA,  #
 
 Pattern = Tuple[int, int, int, int]
 
-__all__ = ["matmul", "matmul_host", "chain", "plan", "sync_status", "workspace_info", "ks_dtype_of", "KsError", "VARIANTS"]
+__all__ = ["matmul", "matmul_host", "matmul_dx", "matmul_dv", "bias_grad", "chain", "butterfly_factorize", "KSLinear",
+           "plan", "sync_status", "workspace_info", "ks_dtype_of", "KsError", "VARIANTS"]
 
 
 def ks_dtype_of(t: torch.Tensor, tf32: bool = False) -> int:
@@ -210,9 +211,10 @@ class _KSLinearFn(torch.autograd.Function):
 class KSLinear(torch.nn.Module):
     """A linear layer whose weight is one KS factor of pattern (a, b, c, d):
     in_features a*c*d, out_features a*b*d, y = x K^T (+ bias, fused into the
-    product's epilogue; its gradient is the column sum of dY, ks_bias_grad).  The values are
-    a parameter of shape (a, d, b, c), drawn N(0, 1/c) (unit-variance outputs
-    for unit-variance inputs).  Leading dimensions of x are flattened."""
+    product's epilogue; its gradient is the column sum of dY, ks_bias_grad).
+    The values are a parameter of shape (a, d, b, c), drawn N(0, 1/c)
+    (unit-variance outputs for unit-variance inputs).  Leading dimensions of x
+    are flattened."""
 
     def __init__(self, pattern: Pattern, bias: bool = False, dtype=torch.float32, device=None):
         super().__init__()
