@@ -174,6 +174,20 @@ def test_host_product_validates_on_the_host(lib):
     assert lib.ks_matmul_host(None, None, 2, 2, 2, 2, 0, None, 0, None) == 0  # batch 0: no-op
 
 
+def test_bias_grad_validates_on_the_host(lib):
+    # dY at P (4 x 8 fp32 = 128 bytes), db elsewhere
+    assert lib.ks_bias_grad(P, 4, 8, None, 0, None) == 1            # null db
+    assert lib.ks_bias_grad(None, 4, 8, P * 8, 0, None) == 1        # null dY with rows to sum
+    assert lib.ks_bias_grad(P, -1, 8, P * 8, 0, None) == 1          # negative batch
+    assert lib.ks_bias_grad(P, 4, 0, P * 8, 0, None) == 1           # empty width
+    assert lib.ks_bias_grad(P, 4, 8, P * 8, 7, None) == 1           # unknown dtype
+    assert lib.ks_bias_grad(P, 1 << 62, 1 << 3, P * 8, 0, None) == 1  # sizes overflow
+    assert lib.ks_bias_grad(P, 4, 8, P + 64, 0, None) == 1          # db inside dY
+    assert b"overlaps" in lib.ks_last_error()
+    assert lib.ks_bias_grad(P, 4, 8, P * 8 + 2, 0, None) == 2       # fp32 db not 4-byte aligned
+    assert lib.ks_bias_grad(P + 1, 4, 8, P * 8, 2, None) == 2       # bf16 dY not 2-byte aligned
+
+
 def test_fma_rate_probe_validates_on_the_host(lib):
     assert lib.ks_fma_rate_probe(None, 4, 16, None) == 1
     assert lib.ks_fma_rate_probe(P, 0, 16, None) == 1
